@@ -1,0 +1,221 @@
+/*
+ * libppattn -- B200 (sm_100a) attention for Parallel Prompting.
+ *
+ * Source of the method: "Read Once, Answer Many: Parallel Prompting for
+ * Shared-Context LLM Inference" (Zhao & Flanigan), project page, section
+ * "How it works", and the arXiv abstract of the same paper.  P independent
+ * questions about one document are decoded as P answer streams of a single
+ * request.  Every decode step reads the document KV once for all P streams,
+ * and a stream-id mask evaluated inside the attention kernel (no dense mask
+ * tensor) keeps each answer conditioned only on the document and on its own
+ * question and answer tokens.  Every stream's positions start right after the
+ * document ("shared positions"), and a decode step has a fixed shape so it
+ * can be captured in a CUDA graph.
+ *
+ * Mask rule implemented by every kernel here (same section, item 1): a query
+ * of stream s at position p sees key j iff
+ *     j is a document key (stream id 0, index < doc_len), or
+ *     sid_j == s  and  pos_j <= p        (own stream, causally earlier or
+ *                                         the query's own token).
+ * The page numbers the document -1; this library numbers it 0 and the answer
+ * streams 1..P (stream id -1 marks an inactive query row).
+ *
+ * Conventions for every entry point
+ *   - Pointers are DEVICE pointers unless their name starts with h_.
+ *   - bf16 tensors are passed as uint16_t bit patterns (IEEE bfloat16).
+ *   - The caller owns and allocates every buffer (KV cache, tags, q, o, lse,
+ *     workspace).  The library allocates no device memory and keeps no
+ *     device state between calls.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream), perform no host synchronisation and no allocation,
+ *     and may be captured into a CUDA graph -- except pp_get_device_status,
+ *     which synchronises.
+ *   - Host-side argument checks return an error before anything is
+ *     launched.  Errors found on the device set bits of the layer's device
+ *     status word (PP_DEV_*), read with pp_get_device_status.
+ *   - Inputs q, k, v, sid, pos are never written.
+ *   - bf16 device pointers must be 16-byte aligned.
+ */
+#ifndef PPATTN_H
+#define PPATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define PP_ABI_VERSION 1
+
+typedef enum pp_status {
+    PP_OK = 0,
+    PP_ERR_INVALID_ARG = 1,     /* NULL / misaligned pointer, negative size   */
+    PP_ERR_UNSUPPORTED = 2,     /* d not in {64,128}, P > P_max, P > 32767    */
+    PP_ERR_CAPACITY = 3,        /* doc_len > doc_cap, workspace too small     */
+    PP_ERR_CUDA = 4,            /* a CUDA launch or driver call failed        */
+    PP_ERR_DEVICE_TIMEOUT = 5   /* reserved for callers mapping PP_DEV_TIMEOUT */
+} pp_status;
+
+/* Bits of the per-layer device status word (sticky; cleared by pp_kv_reset). */
+#define PP_DEV_SEGMENT_OVERFLOW 0x1  /* append: stream segment full, row dropped */
+#define PP_DEV_DOC_OUT_OF_RANGE 0x2  /* append: document position outside cache */
+#define PP_DEV_BAD_STREAM       0x4  /* stream id > P_max, or a document query   */
+#define PP_DEV_TIMEOUT          0x8  /* a bounded in-kernel wait gave up         */
+
+/*
+ * One attention layer's KV cache ("How it works": every KV slot carries a
+ * stream id; the document KV is shared by all streams).
+ *
+ *   k_doc, v_doc  bf16 [H][doc_cap][d]   document block, head-major; document
+ *                                        token i sits at index i (stream id 0,
+ *                                        position i, both implicit).
+ *   k_suf, v_suf  bf16 [P_max][H][S_cap][d]   one segment per answer stream:
+ *                                        stream s (1..P_max) owns index s-1;
+ *                                        its question and answer tokens in
+ *                                        append order.
+ *   sid           int16 [P_max][S_cap]   stream id of every segment slot.
+ *   pos           int32 [P_max][S_cap]   position of every segment slot.
+ *   len           int32 [P_max]          slots in use per segment; slots at or
+ *                                        beyond len are never read.
+ *   status        int32 [1]              device status word (PP_DEV_* bits).
+ */
+typedef struct pp_kv_layer {
+    int32_t H, d, doc_cap, P_max, S_cap;
+    int32_t reserved;
+    uint16_t *k_doc, *v_doc;
+    uint16_t *k_suf, *v_suf;
+    int16_t *sid;
+    int32_t *pos;
+    int32_t *len;
+    int32_t *status;
+} pp_kv_layer;
+
+/*
+ * Options (NULL = all defaults).
+ *   splits                  0 = automatic document split; else the number of
+ *                           CTAs the document pass runs on (>= 1).
+ *   ablation_doc_per_stream 1 = read the document once PER STREAM (one warp
+ *                           per stream and head, no tensor cores) instead of
+ *                           once per step: the batched-requests baseline of the
+ *                           page's "Inside decode step" figure, kept to measure
+ *                           the bytes Parallel Prompting saves.
+ *   debug_inject_timeout    test only: 1 = the document pass's producer skips
+ *                           its first copy, so the consumers' bounded waits
+ *                           expire; the call then sets PP_DEV_TIMEOUT and
+ *                           returns without hanging.
+ *   wait_limit_log2         test only: 0 = default bound on in-kernel waits
+ *                           (about 2^31 clock cycles); else 2^value cycles.
+ */
+typedef struct pp_options {
+    int32_t splits;
+    int32_t ablation_doc_per_stream;
+    int32_t debug_inject_timeout;
+    int32_t wait_limit_log2;
+} pp_options;
+
+/* Human-readable name of a pp_status value. */
+const char *pp_status_str(int32_t status);
+
+/* PP_ABI_VERSION of the loaded library. */
+int32_t pp_abi_version(void);
+
+/* Zero len[] and the status word of a layer (asynchronous). */
+pp_status pp_kv_reset(const pp_kv_layer *layer, void *stream);
+
+/*
+ * Append n rows to the cache ("How it works": each decode step appends one
+ * token per stream; the document is written once as stream 0).
+ *   k, v  bf16 [n][H][d];  sid int16 [n];  pos int32 [n].
+ * Row i with sid 0 is written to document index pos[i] (0 <= pos < doc_cap,
+ * else dropped + PP_DEV_DOC_OUT_OF_RANGE).  Row i with sid s in [1, P_max]
+ * goes to slot len[s-1] + r of segment s-1, where r counts earlier rows of
+ * the same stream in this call; its sid and pos are stored with it, and
+ * len[s-1] advances.  A full segment drops the row and sets
+ * PP_DEV_SEGMENT_OVERFLOW; sid > P_max sets PP_DEV_BAD_STREAM; sid < 0 rows
+ * are skipped.  Two kernel launches; n = 0 launches nothing.
+ */
+pp_status pp_kv_append(const pp_kv_layer *layer, const uint16_t *k, const uint16_t *v,
+                       const int16_t *sid, const int32_t *pos, int32_t n, void *stream);
+
+/*
+ * Workspace bytes pp_decode_attn needs for P query rows (fp32 partial
+ * results of the split document pass and of the suffix pass).  The split
+ * plan depends on the SM count of the CURRENT device: query with the device
+ * that will run the call.  Returns 0 on bad arguments or without a device.
+ */
+size_t pp_decode_workspace_bytes(int32_t P, int32_t H, int32_t d, int32_t doc_len,
+                                 const pp_options *opt);
+
+/*
+ * Decode-step attention ("How it works": one query per stream per step; the
+ * document K/V are read once for all P streams).
+ *   q      bf16 [P][H][d]   query of row i (usually stream i+1's new token)
+ *   q_sid  int16 [P]        stream of row i: 1..P_max, or -1 for an inactive
+ *                           row (its o is 0 and its lse -inf)
+ *   q_pos  int32 [P]        position of row i (shared positions: N + tokens
+ *                           the stream has before this one)
+ *   doc_len (host)          document keys 0..doc_len-1 are visible
+ *   scale                   softmax scale (1/sqrt(d) for the usual model)
+ *   o      bf16 [P][H][d]   output (round-to-nearest-even from fp32)
+ *   lse    fp32 [P][H]      natural-log sum-exp of the scaled scores, or NULL
+ *   ws     workspace of at least pp_decode_workspace_bytes(...) bytes
+ * The stream's own K/V for this step must already be appended.  Rows with
+ * sid 0 (document queries) or sid > P_max get o = 0 and PP_DEV_BAD_STREAM.
+ */
+pp_status pp_decode_attn(const pp_kv_layer *layer, int32_t doc_len, const uint16_t *q,
+                         const int16_t *q_sid, const int32_t *q_pos, int32_t P, float scale,
+                         uint16_t *o, float *lse, void *ws, size_t ws_bytes,
+                         const pp_options *opt, void *stream);
+
+/* Workspace bytes pp_prefill_attn needs for R question rows. */
+size_t pp_prefill_workspace_bytes(int32_t R, int32_t H, int32_t d, int32_t doc_len,
+                                  const pp_options *opt);
+
+/*
+ * Question prefill of all P questions in one call (the page's introductory
+ * figure: the document and all questions go into one sequence, prefilled
+ * once; each question gets its own answer stream that sees only the
+ * document and its own question).
+ *   q       bf16 [R][H][d]  question rows, any order
+ *   q_sid   int16 [R]       stream of each row (1..P_max; -1 = inactive)
+ *   q_pos   int32 [R]       position of each row (N + index in its question)
+ *   o bf16 [R][H][d], lse fp32 [R][H] or NULL, ws as for decode.
+ * The question rows' own K/V must already be appended (pp_kv_append).  Each
+ * row sees the document and the rows of its own stream at positions <= its
+ * own (causal within the question).  Row errors are flagged as for decode.
+ */
+pp_status pp_prefill_attn(const pp_kv_layer *layer, int32_t doc_len, const uint16_t *q,
+                          const int16_t *q_sid, const int32_t *q_pos, int32_t R, float scale,
+                          uint16_t *o, float *lse, void *ws, size_t ws_bytes,
+                          const pp_options *opt, void *stream);
+
+/*
+ * Test aid: evaluate the mask predicate the attention kernels use.
+ *   count_out int32 [nq]: number of keys query i sees (document included).
+ *   mask_out  uint8 [nq][P_max*S_cap] or NULL: 1 where segment slot
+ *             (s-1)*S_cap + t is visible to query i (slots >= len are 0).
+ */
+pp_status pp_debug_visibility(const pp_kv_layer *layer, int32_t doc_len, const int16_t *q_sid,
+                              const int32_t *q_pos, int32_t nq, int32_t *count_out,
+                              uint8_t *mask_out, void *stream);
+
+/*
+ * Test aid (host only, no device needed): the document split the attention
+ * calls use for `rows` query rows, H heads and doc_len keys over `ctas` CTAs.
+ * Writes to host array h_out (h_out_len >= 5 + 2*units entries):
+ *   h_out[0..4] = T (key tiles per unit), units (row groups * H), W (total
+ *   tiles), C (CTAs), max_chunks; then per unit u: h_out[5+2u] = first CTA
+ *   and h_out[6+2u] = last CTA whose tile range covers unit u.
+ */
+pp_status pp_debug_split_plan(int32_t rows, int32_t H, int32_t doc_len, int32_t ctas,
+                              int64_t *h_out, int32_t h_out_len);
+
+/* Copy the layer's device status word to *h_status (synchronises stream). */
+pp_status pp_get_device_status(const pp_kv_layer *layer, int32_t *h_status, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PPATTN_H */

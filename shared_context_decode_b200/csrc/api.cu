@@ -1,0 +1,268 @@
+// C-ABI entry points of libppattn (declared in include/ppattn.h).
+//
+// Host code here validates arguments, derives the document split plan,
+// carves the caller's workspace and launches the kernels in stream order:
+//   decode / prefill:  [document pass] -> suffix pass -> log-sum-exp merge
+// Nothing here allocates device memory or synchronises (except
+// pp_get_device_status), so the calls can be captured in a CUDA graph.
+#include <algorithm>
+#include <atomic>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace {
+
+using pp::Partials;
+using pp::SplitPlan;
+
+constexpr size_t kAlign = 256;
+
+size_t up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned(const void* ptr, size_t a) { return (reinterpret_cast<uintptr_t>(ptr) % a) == 0; }
+
+int sm_count() {
+  static std::atomic<int> cache[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (dev < 64 && cache[dev].load() > 0) return cache[dev].load();
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  if (dev < 64) cache[dev].store(n);
+  return n;
+}
+
+pp_status check_layer(const pp_kv_layer* L) {
+  if (!L) return PP_ERR_INVALID_ARG;
+  if (L->d != 64 && L->d != 128) return PP_ERR_UNSUPPORTED;
+  if (L->P_max < 1 || L->P_max > 32767) return PP_ERR_UNSUPPORTED;
+  if (L->H < 1 || L->doc_cap < 0 || L->S_cap < 1) return PP_ERR_INVALID_ARG;
+  if (L->doc_cap > 0 && (!L->k_doc || !L->v_doc || !aligned(L->k_doc, 16) || !aligned(L->v_doc, 16)))
+    return PP_ERR_INVALID_ARG;
+  if (!L->k_suf || !L->v_suf || !aligned(L->k_suf, 16) || !aligned(L->v_suf, 16))
+    return PP_ERR_INVALID_ARG;
+  if (!L->sid || !L->pos || !L->len || !L->status || !aligned(L->sid, 2) || !aligned(L->pos, 4) ||
+      !aligned(L->len, 4) || !aligned(L->status, 4))
+    return PP_ERR_INVALID_ARG;
+  return PP_OK;
+}
+
+pp_status from_cuda(cudaError_t e) { return e == cudaSuccess ? PP_OK : PP_ERR_CUDA; }
+
+// The document split: see pp::SplitPlan.  `ctas` = CTAs to spread it over.
+SplitPlan make_plan(int rows, int H, int doc_len, int ctas) {
+  SplitPlan p{};
+  p.T = (doc_len + pp::kBN - 1) / pp::kBN;
+  p.units = ((rows + pp::kGroupRows - 1) / pp::kGroupRows) * H;
+  p.W = (int64_t)p.units * p.T;
+  if (p.W == 0 || ctas < 1) {
+    p.C = 0;
+    p.max_chunks = 0;
+    return p;
+  }
+  p.C = (int32_t)std::min<int64_t>(ctas, p.W);
+  int mc = 1;
+  for (int u = 0; u < p.units; ++u) {
+    const int n = pp::plan_cta_of(p, (int64_t)u * p.T + p.T - 1) - pp::plan_cta_of(p, (int64_t)u * p.T) + 1;
+    mc = std::max(mc, n);
+  }
+  p.max_chunks = mc;
+  return p;
+}
+
+// The ablation reads the whole document per row: one chunk per unit.
+SplitPlan ablation_plan(int rows, int H, int doc_len) {
+  SplitPlan p{};
+  p.units = ((rows + pp::kGroupRows - 1) / pp::kGroupRows) * H;
+  p.T = doc_len > 0 ? 1 : 0;
+  p.W = (int64_t)p.units * p.T;
+  p.C = (int32_t)p.W;
+  p.max_chunks = p.W > 0 ? 1 : 0;
+  return p;
+}
+
+SplitPlan plan_for(int rows, int H, int doc_len, const pp_options* opt) {
+  if (opt && opt->ablation_doc_per_stream) return ablation_plan(rows, H, doc_len);
+  const int ctas = (opt && opt->splits > 0) ? opt->splits : sm_count();
+  return make_plan(rows, H, doc_len, ctas);
+}
+
+struct WsLayout {
+  size_t doc_o, doc_ml, suf_o, suf_ml, total;
+};
+
+WsLayout ws_layout(int rows, int H, int d, const SplitPlan& p) {
+  WsLayout w;
+  const size_t slots = (size_t)p.units * p.max_chunks * pp::kGroupRows;
+  w.doc_o = 0;
+  w.doc_ml = w.doc_o + up(slots * d * sizeof(float));
+  w.suf_o = w.doc_ml + up(slots * 2 * sizeof(float));
+  w.suf_ml = w.suf_o + up((size_t)rows * H * d * sizeof(float));
+  w.total = w.suf_ml + up((size_t)rows * H * 2 * sizeof(float));
+  return w;
+}
+
+Partials carve(void* ws, const WsLayout& w) {
+  uint8_t* b = static_cast<uint8_t*>(ws);
+  Partials p;
+  p.doc_o = reinterpret_cast<float*>(b + w.doc_o);
+  p.doc_ml = reinterpret_cast<float*>(b + w.doc_ml);
+  p.suf_o = reinterpret_cast<float*>(b + w.suf_o);
+  p.suf_ml = reinterpret_cast<float*>(b + w.suf_ml);
+  return p;
+}
+
+long long wait_limit(const pp_options* opt) {
+  const int lg = (opt && opt->wait_limit_log2 > 0) ? std::min(opt->wait_limit_log2, 40) : 31;
+  return 1LL << lg;
+}
+
+// Shared body of decode and prefill attention.
+pp_status attend(const pp_kv_layer* L, int32_t doc_len, const uint16_t* q, const int16_t* q_sid,
+                 const int32_t* q_pos, int32_t rows, float scale, uint16_t* o, float* lse, void* ws,
+                 size_t ws_bytes, const pp_options* opt, void* stream) {
+  pp_status s = check_layer(L);
+  if (s != PP_OK) return s;
+  if (rows < 0 || doc_len < 0) return PP_ERR_INVALID_ARG;
+  if (doc_len > L->doc_cap) return PP_ERR_CAPACITY;
+  if (rows == 0) return PP_OK;
+  if (!q || !q_sid || !q_pos || !o || !aligned(q, 16) || !aligned(o, 16) || !aligned(q_sid, 2) ||
+      !aligned(q_pos, 4) || (lse && !aligned(lse, 4)))
+    return PP_ERR_INVALID_ARG;
+  if (!(scale == scale)) return PP_ERR_INVALID_ARG;
+  const SplitPlan plan = plan_for(rows, L->H, doc_len, opt);
+  const bool has_doc = doc_len > 0;
+  if (has_doc && plan.C < 1) return PP_ERR_CUDA;  // no device to size the split for
+  const WsLayout w = ws_layout(rows, L->H, L->d, plan);
+  if (!ws || !aligned(ws, kAlign)) return PP_ERR_INVALID_ARG;
+  if (ws_bytes < w.total) return PP_ERR_CAPACITY;
+  const Partials part = carve(ws, w);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (has_doc) {
+    cudaError_t e;
+    if (opt && opt->ablation_doc_per_stream)
+      e = pp::launch_doc_per_stream(*L, doc_len, q, q_sid, rows, scale, plan.max_chunks, part, st);
+    else
+      e = pp::launch_doc_pass_tc(*L, doc_len, q, rows, scale, plan, part, wait_limit(opt),
+                                 opt ? opt->debug_inject_timeout : 0, st);
+    if (e != cudaSuccess) return PP_ERR_CUDA;
+  }
+  if ((s = from_cuda(pp::launch_suffix_pass(*L, q, q_sid, q_pos, rows, scale, part, st))) != PP_OK)
+    return s;
+  return from_cuda(pp::launch_lse_merge(rows, L->H, L->d, L->P_max, plan, has_doc, q_sid, part, o,
+                                        lse, st));
+}
+
+size_t workspace(int32_t rows, int32_t H, int32_t d, int32_t doc_len, const pp_options* opt) {
+  if (rows < 0 || H < 1 || (d != 64 && d != 128) || doc_len < 0) return 0;
+  const SplitPlan plan = plan_for(rows, H, doc_len, opt);
+  if (doc_len > 0 && plan.C < 1) return 0;
+  return ws_layout(rows, H, d, plan).total;
+}
+
+}  // namespace
+
+extern "C" {
+
+#define PP_API __attribute__((visibility("default")))
+
+PP_API const char* pp_status_str(int32_t status) {
+  switch (status) {
+    case PP_OK: return "PP_OK";
+    case PP_ERR_INVALID_ARG: return "PP_ERR_INVALID_ARG";
+    case PP_ERR_UNSUPPORTED: return "PP_ERR_UNSUPPORTED";
+    case PP_ERR_CAPACITY: return "PP_ERR_CAPACITY";
+    case PP_ERR_CUDA: return "PP_ERR_CUDA";
+    case PP_ERR_DEVICE_TIMEOUT: return "PP_ERR_DEVICE_TIMEOUT";
+    default: return "PP_ERR_UNKNOWN";
+  }
+}
+
+PP_API int32_t pp_abi_version(void) { return PP_ABI_VERSION; }
+
+PP_API pp_status pp_kv_reset(const pp_kv_layer* layer, void* stream) {
+  pp_status s = check_layer(layer);
+  if (s != PP_OK) return s;
+  return from_cuda(pp::launch_kv_reset(*layer, static_cast<cudaStream_t>(stream)));
+}
+
+PP_API pp_status pp_kv_append(const pp_kv_layer* layer, const uint16_t* k, const uint16_t* v,
+                       const int16_t* sid, const int32_t* pos, int32_t n, void* stream) {
+  pp_status s = check_layer(layer);
+  if (s != PP_OK) return s;
+  if (n < 0) return PP_ERR_INVALID_ARG;
+  if (n == 0) return PP_OK;
+  if (!k || !v || !sid || !pos || !aligned(k, 16) || !aligned(v, 16) || !aligned(sid, 2) ||
+      !aligned(pos, 4))
+    return PP_ERR_INVALID_ARG;
+  return from_cuda(pp::launch_kv_append(*layer, k, v, sid, pos, n, static_cast<cudaStream_t>(stream)));
+}
+
+PP_API size_t pp_decode_workspace_bytes(int32_t P, int32_t H, int32_t d, int32_t doc_len,
+                                 const pp_options* opt) {
+  return workspace(P, H, d, doc_len, opt);
+}
+
+PP_API size_t pp_prefill_workspace_bytes(int32_t R, int32_t H, int32_t d, int32_t doc_len,
+                                  const pp_options* opt) {
+  return workspace(R, H, d, doc_len, opt);
+}
+
+PP_API pp_status pp_decode_attn(const pp_kv_layer* layer, int32_t doc_len, const uint16_t* q,
+                         const int16_t* q_sid, const int32_t* q_pos, int32_t P, float scale,
+                         uint16_t* o, float* lse, void* ws, size_t ws_bytes, const pp_options* opt,
+                         void* stream) {
+  if (layer && P > layer->P_max) return PP_ERR_UNSUPPORTED;
+  return attend(layer, doc_len, q, q_sid, q_pos, P, scale, o, lse, ws, ws_bytes, opt, stream);
+}
+
+PP_API pp_status pp_prefill_attn(const pp_kv_layer* layer, int32_t doc_len, const uint16_t* q,
+                          const int16_t* q_sid, const int32_t* q_pos, int32_t R, float scale,
+                          uint16_t* o, float* lse, void* ws, size_t ws_bytes,
+                          const pp_options* opt, void* stream) {
+  return attend(layer, doc_len, q, q_sid, q_pos, R, scale, o, lse, ws, ws_bytes, opt, stream);
+}
+
+PP_API pp_status pp_debug_visibility(const pp_kv_layer* layer, int32_t doc_len, const int16_t* q_sid,
+                              const int32_t* q_pos, int32_t nq, int32_t* count_out,
+                              uint8_t* mask_out, void* stream) {
+  pp_status s = check_layer(layer);
+  if (s != PP_OK) return s;
+  if (nq < 0 || doc_len < 0) return PP_ERR_INVALID_ARG;
+  if (doc_len > layer->doc_cap) return PP_ERR_CAPACITY;
+  if (nq == 0) return PP_OK;
+  if (!q_sid || !q_pos || !count_out) return PP_ERR_INVALID_ARG;
+  return from_cuda(pp::launch_visibility(*layer, doc_len, q_sid, q_pos, nq, count_out, mask_out,
+                                         static_cast<cudaStream_t>(stream)));
+}
+
+PP_API pp_status pp_debug_split_plan(int32_t rows, int32_t H, int32_t doc_len, int32_t ctas,
+                              int64_t* h_out, int32_t h_out_len) {
+  if (rows < 0 || H < 1 || doc_len < 0 || ctas < 1 || !h_out) return PP_ERR_INVALID_ARG;
+  const SplitPlan p = make_plan(rows, H, doc_len, ctas);
+  if (h_out_len < 5 + 2 * (int64_t)p.units) return PP_ERR_CAPACITY;
+  h_out[0] = p.T;
+  h_out[1] = p.units;
+  h_out[2] = p.W;
+  h_out[3] = p.C;
+  h_out[4] = p.max_chunks;
+  for (int u = 0; u < p.units; ++u) {
+    h_out[5 + 2 * u] = p.W ? pp::plan_cta_of(p, (int64_t)u * p.T) : 0;
+    h_out[6 + 2 * u] = p.W ? pp::plan_cta_of(p, (int64_t)u * p.T + p.T - 1) : -1;
+  }
+  return PP_OK;
+}
+
+PP_API pp_status pp_get_device_status(const pp_kv_layer* layer, int32_t* h_status, void* stream) {
+  pp_status s = check_layer(layer);
+  if (s != PP_OK) return s;
+  if (!h_status) return PP_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(h_status, layer->status, sizeof(int32_t), cudaMemcpyDeviceToHost, st) !=
+      cudaSuccess)
+    return PP_ERR_CUDA;
+  return from_cuda(cudaStreamSynchronize(st));
+}
+
+}  // extern "C"

@@ -1,0 +1,125 @@
+"""C-ABI checks that need no GPU: the library loads, exports every entry
+point include/ppattn.h declares, rejects bad arguments on the host before
+any launch, and plans the document split correctly."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from shared_context_decode_b200 import build as ppbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def pp():
+    ppbuild.build()
+    from shared_context_decode_b200 import ppattn
+    return ppattn
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "ppattn.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(pp_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_header_declares_the_three_calls():
+    names = declared_functions()
+    for n in ("pp_kv_append", "pp_decode_attn", "pp_prefill_attn"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(pp):
+    lib = ctypes.CDLL(pp.LIB_PATH)
+    names = declared_functions()
+    assert len(names) >= 10
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in include/ppattn.h but not exported"
+    assert set(names) == set(pp.EXPORTED)
+
+
+def test_status_strings_and_version(pp):
+    assert pp.abi_version() == 1
+    assert pp.status_str(0) == "PP_OK"
+    assert pp.status_str(3) == "PP_ERR_CAPACITY"
+    assert pp.status_str(99) == "PP_ERR_UNKNOWN"
+
+
+def fake_layer(pp, **kw):
+    """A descriptor with plausible aligned (never dereferenced) addresses."""
+    base = dict(H=4, d=128, doc_cap=1024, P_max=8, S_cap=64, reserved=0,
+                k_doc=0x10000, v_doc=0x20000, k_suf=0x30000, v_suf=0x40000,
+                sid=0x50000, pos=0x60000, len=0x70000, status=0x80000)
+    base.update(kw)
+    return pp.LayerStruct(**base)
+
+
+def call_decode(pp, L, doc_len=10, P=4, ws_bytes=1 << 30, opt=None, q=0x90000):
+    return pp._decode(ctypes.byref(L), doc_len, q, 0xA0000, 0xB0000, P, 0.1, 0xC0000, None,
+                      0xD0000, ws_bytes, None if opt is None else ctypes.byref(opt), None)
+
+
+def test_host_validation_codes(pp):
+    L = fake_layer(pp)
+    # layer checks
+    assert pp._kv_reset(None, None) == pp.PP_ERR_INVALID_ARG
+    assert call_decode(pp, fake_layer(pp, d=96)) == pp.PP_ERR_UNSUPPORTED
+    assert call_decode(pp, fake_layer(pp, P_max=0)) == pp.PP_ERR_UNSUPPORTED
+    assert call_decode(pp, fake_layer(pp, P_max=40000)) == pp.PP_ERR_UNSUPPORTED
+    assert call_decode(pp, fake_layer(pp, k_suf=0x30008)) == pp.PP_ERR_INVALID_ARG
+    assert call_decode(pp, fake_layer(pp, len=0)) == pp.PP_ERR_INVALID_ARG
+    # call checks
+    assert call_decode(pp, L, P=9) == pp.PP_ERR_UNSUPPORTED           # P > P_max
+    assert call_decode(pp, L, doc_len=1025) == pp.PP_ERR_CAPACITY     # doc_len > doc_cap
+    assert call_decode(pp, L, doc_len=-1) == pp.PP_ERR_INVALID_ARG
+    assert call_decode(pp, L, q=0x90004) == pp.PP_ERR_INVALID_ARG     # misaligned q
+    assert call_decode(pp, L, P=0) == pp.PP_OK                        # empty: nothing launched
+    opt = pp.Options(splits=4)
+    assert call_decode(pp, L, ws_bytes=16, opt=opt) == pp.PP_ERR_CAPACITY
+    # append
+    assert pp._kv_append(ctypes.byref(L), 0x1000, 0x2000, 0x3000, 0x4000, -1, None) == \
+        pp.PP_ERR_INVALID_ARG
+    assert pp._kv_append(ctypes.byref(L), 0x1000, 0x2000, 0x3000, 0x4000, 0, None) == pp.PP_OK
+    assert pp._kv_append(ctypes.byref(L), 0x1008, 0x2000, 0x3000, 0x4000, 3, None) == \
+        pp.PP_ERR_INVALID_ARG
+    # prefill
+    assert pp._prefill(ctypes.byref(L), 2000, 0x90000, 0xA0000, 0xB0000, 5, 0.1, 0xC0000, None,
+                       0xD0000, 1 << 30, None, None) == pp.PP_ERR_CAPACITY
+    # visibility
+    assert pp._visibility(ctypes.byref(L), 5, 0x1000, 0x2000, -1, 0x3000, None, None) == \
+        pp.PP_ERR_INVALID_ARG
+
+
+def test_workspace_sizes_with_explicit_split(pp):
+    opt = pp.Options(splits=148)
+    ws = pp.decode_workspace_bytes(256, 32, 128, 16384, opt)
+    plan = pp.split_plan(256, 32, 16384, 148)
+    slots = plan["units"] * plan["max_chunks"] * 256
+    expect = slots * 128 * 4 + slots * 2 * 4 + 256 * 32 * 128 * 4 + 256 * 32 * 2 * 4
+    assert ws == expect
+    assert pp.decode_workspace_bytes(4, 4, 96, 10, opt) == 0
+    # no document: only the suffix partials
+    assert pp.decode_workspace_bytes(8, 2, 64, 0, opt) == 8 * 2 * 64 * 4 + 256
+
+
+@pytest.mark.parametrize("rows,H,doc_len,ctas", [
+    (256, 32, 16384, 148), (64, 32, 8192, 148), (8192, 32, 12000, 148), (4, 4, 256, 148),
+    (200, 4, 1000, 3), (300, 2, 300, 7), (1, 1, 1, 148), (256, 32, 16384, 1), (130, 3, 129, 5)])
+def test_split_plan_invariants(pp, rows, H, doc_len, ctas):
+    p = pp.split_plan(rows, H, doc_len, ctas)
+    T = -(-doc_len // 128)
+    units = -(-rows // 256) * H
+    assert p["T"] == T and p["units"] == units and p["W"] == units * T
+    assert p["C"] == min(ctas, units * T)
+    W, C = p["W"], p["C"]
+    begin = [c * W // C for c in range(C + 1)]
+    sizes = [begin[c + 1] - begin[c] for c in range(C)]
+    assert min(sizes) >= W // C and max(sizes) <= -(-W // C)    # balanced to one tile
+    for u, (c0, c1) in enumerate(p["chunks"]):
+        # the CTAs listed are exactly those whose range meets the unit's tiles
+        meets = [c for c in range(C) if begin[c] < (u + 1) * T and begin[c + 1] > u * T]
+        assert (c0, c1) == (meets[0], meets[-1])
+        assert c1 - c0 + 1 <= p["max_chunks"]
+    assert p["max_chunks"] == max(c1 - c0 + 1 for c0, c1 in p["chunks"])

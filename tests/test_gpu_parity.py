@@ -1,0 +1,128 @@
+"""GPU parity: the C-ABI path against the fp64 oracle, element by element.
+
+Small cases are compared in full and span several document tiles, both M
+tiles of a row group, two row groups, ragged tails and forced split counts
+that make CTAs cross head boundaries; the named full-size workloads are
+compared on sampled rows (all heads, all d) in the launch configuration the
+bench uses.
+"""
+import numpy as np
+import pytest
+import torch
+
+from shared_context_decode_b200 import workloads as wl
+from tests import gpu_util as gu
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def decode_case(W, l=0, opt=None, rows=None, with_lse=True):
+    m = gu.pp()
+    L = W.layer(l)
+    layer = gu.load_decode(W, L, DEV)
+    lse = torch.empty((W.P, W.H), dtype=torch.float32, device=DEV) if with_lse else None
+    o = m.decode_attn(layer, W.N, L.q, L.q_sid, L.q_pos, W.scale, lse=lse, opt=opt)
+    torch.cuda.synchronize()
+    assert m.device_status(layer) == 0
+    o_ref, lse_ref, _ = gu.oracle_decode(W, L, rows)
+    sel = slice(None) if rows is None else rows
+    return gu.compare(o[sel], None if lse is None else lse[sel], o_ref, lse_ref, W.name)
+
+
+def test_tiny_config_full():
+    decode_case(wl.make_decode("tiny", device=DEV))
+
+
+@pytest.mark.parametrize("splits", [0, 1, 3, 7])
+def test_ragged_two_mtiles_split_variants(splits):
+    # 8 key tiles with a 104-key tail, 200 rows = 128 + 72, 4 heads
+    W = wl.make_decode(layers=1, H=4, d=128, N=1000, P=200, q=(1, 20), a=(0, 10), seed=1,
+                       device=DEV)
+    opt = gu.pp().Options(splits=splits) if splits else None
+    decode_case(W, opt=opt)
+
+
+def test_two_row_groups():
+    W = wl.make_decode(layers=1, H=2, d=128, N=300, P=300, q=(1, 9), a=(0, 4), seed=2,
+                       device=DEV)
+    decode_case(W, opt=gu.pp().Options(splits=5))
+
+
+def test_d64_two_mtiles():
+    W = wl.make_decode(layers=1, H=3, d=64, N=777, P=130, q=(2, 12), a=(0, 7), seed=3, device=DEV)
+    decode_case(W)
+
+
+def test_small_p_single_row():
+    W = wl.make_decode(layers=1, H=2, d=128, N=129, P=1, q=(3, 3), a=(1, 1), seed=4, device=DEV)
+    decode_case(W)
+
+
+def test_no_document():
+    W = wl.make_decode(layers=1, H=2, d=128, N=0, P=5, q=(1, 6), a=(0, 3), seed=5, device=DEV)
+    decode_case(W)
+
+
+def test_ablation_doc_per_stream_matches():
+    W = wl.make_decode(layers=1, H=4, d=128, N=1000, P=40, q=(1, 20), a=(0, 10), seed=6,
+                       device=DEV)
+    decode_case(W, opt=gu.pp().Options(ablation_doc_per_stream=1))
+
+
+def test_inactive_rows_are_zero():
+    m = gu.pp()
+    W = wl.make_decode(layers=1, H=2, d=128, N=260, P=20, q=(1, 5), a=(0, 3), seed=7, device=DEV)
+    active = np.arange(W.P) % 3 != 1
+    L = W.layer(0, active=active)
+    layer = gu.load_decode(W, L, DEV)
+    lse = torch.empty((W.P, W.H), dtype=torch.float32, device=DEV)
+    o = m.decode_attn(layer, W.N, L.q, L.q_sid, L.q_pos, W.scale, lse=lse)
+    torch.cuda.synchronize()
+    o_ref, lse_ref, _ = gu.oracle_decode(W, L)
+    gu.compare(o, lse, o_ref, lse_ref, "inactive")
+    assert torch.all(o[torch.from_numpy(~active).to(DEV)] == 0)
+    assert torch.all(torch.isinf(lse[torch.from_numpy(~active).to(DEV)]))
+
+
+def test_doc_pass_stays_in_segment_when_other_streams_longer():
+    # Streams with very different suffix lengths; the mask must not leak.
+    W = wl.make_decode(layers=1, H=2, d=128, N=400, P=9, q=(1, 60), a=(0, 60), seed=8, device=DEV)
+    decode_case(W)
+
+
+@pytest.mark.parametrize("name", ["doc8k_p64", "doc16k_p256"])
+def test_full_size_sampled(name):
+    W = wl.make_decode(name, device=DEV)
+    rng = np.random.default_rng(0)
+    rows = np.sort(rng.choice(W.P, size=min(W.P, 12), replace=False))
+    for l in (0, W.layers - 1):
+        decode_case(W, l=l, rows=rows)
+
+
+def test_prefill_small_full():
+    m = gu.pp()
+    W = wl.make_prefill(layers=1, H=2, d=128, N=700, P=12, q=(1, 40), seed=9, device=DEV)
+    L = W.layer(0)
+    layer = gu.load_prefill(W, L, DEV)
+    lse = torch.empty((W.R, W.H), dtype=torch.float32, device=DEV)
+    o = m.prefill_attn(layer, W.N, L.q, L.sid, L.pos, W.scale, lse=lse)
+    torch.cuda.synchronize()
+    assert m.device_status(layer) == 0
+    o_ref, lse_ref, _ = gu.oracle_prefill(W, L)
+    gu.compare(o, lse, o_ref, lse_ref, "prefill small")
+
+
+def test_prefill_full_size_sampled():
+    m = gu.pp()
+    W = wl.make_prefill("prefill_doc12k_p256", device=DEV)
+    L = W.layer(0)
+    layer = gu.load_prefill(W, L, DEV)
+    lse = torch.empty((W.R, W.H), dtype=torch.float32, device=DEV)
+    o = m.prefill_attn(layer, W.N, L.q, L.sid, L.pos, W.scale, lse=lse)
+    torch.cuda.synchronize()
+    assert m.device_status(layer) == 0
+    rng = np.random.default_rng(1)
+    rows = np.sort(rng.choice(W.R, size=16, replace=False))
+    o_ref, lse_ref, _ = gu.oracle_prefill(W, L, rows)
+    gu.compare(o[rows], lse[rows], o_ref, lse_ref, "prefill full")
