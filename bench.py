@@ -1,0 +1,440 @@
+"""Benchmark of the Parallel Prompting decode step on B200.
+
+A step is one decode step of a request with P answer streams over all L
+layers: per layer, append every stream's new K/V (pp_kv_append), then the
+decode attention (pp_decode_attn: document pass on the tensor cores, suffix
+pass, log-sum-exp merge).  The step is captured once as a CUDA graph and
+replayed; the KV cache is restored to its pre-step lengths at the start of
+every step, so each step does identical work on identical inputs.
+
+Default workload: doc 16384 tokens, P = 256 streams, H = 32, d = 128,
+32 layers, question lengths U[16,48], cached answers U[0,63] (bf16, seeded
+synthetic data).  The document KV one step reads (8.6 GB) is far larger than
+the 126 MB L2, so no flush is needed between steps.
+
+Output: one JSON line on rank 0 (see the keys in main()).  Multi-GPU
+(torchrun): every rank runs an independent replica (weak scaling, no data
+collective); time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decode-attn stream-tokens/s"
+UNIT = "stream-tokens/s"
+
+
+# ------------------------------------------------------------ distributed --
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def reduce_max(x: float, world: int, device) -> float:
+    """Max over ranks of a per-rank float (a timing)."""
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def reduce_sum(x: float, world: int, device) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def aggregate(units_per_rank: float, ms_per_step_rank: float, world: int, device):
+    """Whole-job throughput: units of all ranks / the slowest rank's time."""
+    ms = reduce_max(ms_per_step_rank, world, device)
+    units = reduce_sum(units_per_rank, world, device)
+    return units / (ms / 1e3), ms
+
+
+# ---------------------------------------------------------------- clocks ---
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms; summary()
+    keeps the samples taken inside [t_start, t_end] (host clock)."""
+    Q = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv")
+        self.t_start = self.t_end = None
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.Q}", "--format=csv",
+                 "-lms", "200"], stdout=self.f, stderr=subprocess.DEVNULL)
+            time.sleep(0.5)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            time.sleep(0.3)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.f.close()
+
+    def mark(self, which: str):
+        setattr(self, "t_" + which, time.time())
+
+    def summary(self):
+        import datetime
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        mhz, mx, reasons, seen = [], None, set(), 0
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path).read().splitlines()[1:]:
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 10:
+                continue
+            try:
+                ts = datetime.datetime.strptime(f[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                sm, mxv = float(f[2].split()[0]), float(f[3].split()[0])
+            except ValueError:
+                continue
+            seen += 1
+            if self.t_start is not None and not (self.t_start - 0.25 <= ts <= self.t_end + 0.25):
+                continue
+            mhz.append(sm)
+            mx = mxv
+            for n, v in zip(names, f[6:10]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": float(np.median(mhz)) if mhz else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(mhz), "samples_total": seen}
+
+
+# --------------------------------------------------------------- workload --
+class DecodeStep:
+    """Device-resident cache of all layers, the step's inputs, and the
+    captured CUDA graph of one decode step."""
+
+    def __init__(self, name: str, layers: int, device, seed: int = 0):
+        from shared_context_decode_b200 import ppattn as pp
+        from shared_context_decode_b200 import workloads as wl
+        self.pp = pp
+        self.W = W = wl.make_decode(name, seed=seed, device=device)
+        self.layers = layers
+        self.device = device
+        self.S_cap = int(math.ceil(W.S_need / 16) * 16)
+        self.len_all = torch.zeros((layers, W.P), dtype=torch.int32, device=device)
+        self.cache, self.inp = [], []
+        for l in range(layers):
+            L = W.layer(l)
+            kv = pp.KVLayer(W.H, W.d, W.N, W.P, self.S_cap, device, len_buf=self.len_all[l])
+            pp.kv_append(kv, L.doc_k, L.doc_v, torch.zeros(W.N, dtype=torch.int16, device=device),
+                         torch.arange(W.N, dtype=torch.int32, device=device))
+            pp.kv_append(kv, L.suf_k, L.suf_v, L.suf_sid, L.suf_pos)
+            self.cache.append(kv)
+            self.inp.append(dict(k=L.new_k, v=L.new_v, q=L.q, sid=L.q_sid, pos=L.q_pos,
+                                 o=torch.empty_like(L.q)))
+            del L
+        torch.cuda.synchronize()
+        self.len0 = self.len_all.clone()
+        self.ws = pp.workspace(pp.decode_workspace_bytes(W.P, W.H, W.d, W.N), device)
+        self.graph = None
+
+    def run_eager(self, opt=None, layer_events=None):
+        pp = self.pp
+        self.len_all.copy_(self.len0)
+        for l in range(self.layers):
+            x = self.inp[l]
+            pp.kv_append(self.cache[l], x["k"], x["v"], x["sid"], x["pos"])
+            if layer_events is not None:
+                opt.set_events(layer_events[l])
+            pp.decode_attn(self.cache[l], self.W.N, x["q"], x["sid"], x["pos"], self.W.scale,
+                           o=x["o"], ws=self.ws, opt=opt)
+
+    def capture(self):
+        self.run_eager()           # warm: per-device setup happens outside the capture
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        s = torch.cuda.Stream(self.device)
+        s.wait_stream(torch.cuda.current_stream(self.device))
+        with torch.cuda.stream(s):
+            with torch.cuda.graph(g, stream=s):
+                self.run_eager()
+        torch.cuda.current_stream(self.device).wait_stream(s)
+        torch.cuda.synchronize()
+        self.graph = g
+
+    def replay(self):
+        self.graph.replay()
+
+    def kernels_per_step(self) -> int:
+        # per layer: append (rows + lengths) 2, document pass 1, suffix pass + merge 1
+        return self.layers * 4
+
+    def check_status(self):
+        for kv in self.cache:
+            st = self.pp.device_status(kv)
+            if st:
+                raise RuntimeError(f"device status {st:#x}")
+
+
+def doc_pass_algorithmic(W):
+    """Algorithmic bytes and FLOPs of one document-pass launch (one layer):
+    every document K and V byte read once; S = Q K^T and O = P V over all
+    P rows."""
+    bytes_ = 2 * W.N * W.H * W.d * 2
+    flops = 4 * W.P * W.N * W.d * W.H
+    return bytes_, flops
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(hbm=d["hbm_gbs"], bf16=d["bf16_tflops"],
+                    bf16_sustained=d.get("bf16_tflops_sustained", d["bf16_tflops"]),
+                    source="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
+
+
+def measure_doc_pass(step: DecodeStep, reps: int):
+    """Average device duration of the document-pass kernel, from CUDA events
+    the library records around it on the launching stream, over `reps`
+    eager passes of all layers."""
+    pp = step.pp
+    opt = pp.Options()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(step.layers)]
+    durs = {"doc": [], "suffix": []}
+    for _ in range(reps):
+        step.run_eager(opt=opt, layer_events=evs)
+        torch.cuda.synchronize()
+        for e in evs:
+            durs["doc"].append(e[0].elapsed_time(e[1]))
+            durs["suffix"].append(e[1].elapsed_time(e[2]))
+    return {k: float(np.mean(v)) for k, v in durs.items()}
+
+
+# ------------------------------------------------------------ CPU oracle ---
+def oracle_sample(W, target_s: float, layer: int = 0):
+    """Time the fp64 oracle on a bounded sample of the workload: all heads
+    of `n` stream rows of one layer, n grown until the sample takes about
+    target_s seconds.  Returns (stream-tokens/s for a full L-layer step,
+    threads, description)."""
+    import oracle
+    from shared_context_decode_b200.workloads import bf16_bits
+    L = W.layer(layer)
+    k = np.concatenate([bf16_bits(L.doc_k), bf16_bits(L.suf_k), bf16_bits(L.new_k)])
+    v = np.concatenate([bf16_bits(L.doc_v), bf16_bits(L.suf_v), bf16_bits(L.new_v)])
+    ks = np.concatenate([np.zeros(W.N, np.int32), L.suf_sid.cpu().numpy().astype(np.int32),
+                         L.q_sid.cpu().numpy().astype(np.int32)])
+    kp = np.concatenate([np.arange(W.N, dtype=np.int32), L.suf_pos.cpu().numpy(),
+                         L.q_pos.cpu().numpy()])
+    q, qs, qp = bf16_bits(L.q), L.q_sid.cpu().numpy(), L.q_pos.cpu().numpy()
+    n, spent = 1, 0.0
+    while True:
+        t0 = time.perf_counter()
+        oracle.masked_attention(q[:n], qs[:n], qp[:n], k, v, ks, kp, W.scale)
+        spent = time.perf_counter() - t0
+        if spent >= target_s or n >= W.P:
+            break
+        n = min(W.P, max(n + 1, int(n * min(4.0, 1.2 * target_s / max(spent, 1e-3)))))
+    per_row_layer = spent / n
+    value = 1.0 / (per_row_layer * W.layers)
+    desc = (f"layer {layer}: {n} of {W.P} stream rows x all {W.H} heads in {spent:.1f} s; "
+            f"per-row cost scaled to {W.layers} layers")
+    return value, oracle.num_threads(), desc
+
+
+def reference_arm(args, world, rank):
+    """--impl reference: the oracle as it stands, on the host cores."""
+    if rank != 0:
+        return
+    from shared_context_decode_b200 import workloads as wl
+    W = wl.make_decode(args.workload, device="cpu")
+    vals = []
+    for i in range(args.warmup + args.steps):
+        val, threads, desc = oracle_sample(W, args.ref_seconds, layer=i % W.layers)
+        if i >= args.warmup:
+            vals.append(val)
+    value = float(np.mean(vals))
+    ms = W.P / value * 1e3
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": args.workload, "layers": W.layers, "H": W.H, "d": W.d,
+                       "doc_tokens": W.N, "streams": W.P},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ main ---
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="doc16k_p256")
+    ap.add_argument("--layers", type=int, default=0, help="0 = the workload's layer count")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="CPU-baseline sample budget (0 = skip)")
+    ap.add_argument("--ref-seconds", type=float, default=10.0)
+    ap.add_argument("--roofline-reps", type=int, default=3)
+    args = ap.parse_args()
+    world, rank, local = dist_env()
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl" if torch.cuda.is_available() else "gloo",
+                                timeout=datetime.timedelta(seconds=300))
+    if args.impl == "reference":
+        reference_arm(args, world, rank)
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return
+    assert args.warmup >= 3, "at least 3 warm-up steps"
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    from shared_context_decode_b200 import workloads as wl
+    nl = args.layers or wl.CONFIGS[args.workload]["layers"]
+    step = DecodeStep(args.workload, nl, dev)
+    W = step.W
+    step.capture()
+
+    # ---- device-resident throughput: graph replays
+    for _ in range(args.warmup):
+        step.replay()
+    torch.cuda.synchronize()
+    barrier(world)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clocks:
+        torch.cuda.synchronize()
+        clocks.mark("start")
+        t0.record()
+        for _ in range(args.steps):
+            step.replay()
+        t1.record()
+        torch.cuda.synchronize()
+        clocks.mark("end")
+    barrier(world)
+    ms_rank = t0.elapsed_time(t1) / args.steps
+    step.check_status()
+    value, ms = aggregate(W.P, ms_rank, world, dev)
+
+    # ---- end to end through the C ABI with host buffers
+    names = ("k", "v", "q", "sid", "pos")
+    host_in = [{n: step.inp[l][n].cpu().pin_memory() for n in names} for l in range(nl)]
+    host_out = [torch.empty_like(step.inp[l]["o"], device="cpu").pin_memory() for l in range(nl)]
+    h2d = sum(t.numel() * t.element_size() for d in host_in for t in d.values())
+    d2h = sum(t.numel() * t.element_size() for t in host_out)
+
+    def e2e_step():
+        for l in range(nl):
+            for n in names:
+                step.inp[l][n].copy_(host_in[l][n], non_blocking=True)
+        step.replay()
+        for l in range(nl):
+            host_out[l].copy_(step.inp[l]["o"], non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ek = max(3, args.steps // 2)
+    e0.record()
+    for _ in range(ek):
+        e2e_step()
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_value, e2e_ms = aggregate(W.P, e0.elapsed_time(e1) / ek, world, dev)
+
+    # ---- roofline of the dominant kernel (document pass), live CUDA events
+    durs = measure_doc_pass(step, args.roofline_reps)
+    peaks = load_peaks()
+    b, f = doc_pass_algorithmic(W)
+    t_doc = durs["doc"] * 1e-3
+    gbs, tfs = b / t_doc / 1e9, f / t_doc / 1e12
+    t_hbm, t_tc = b / (peaks["hbm"] * 1e9), f / (peaks["bf16_sustained"] * 1e12)
+    if t_tc > t_hbm:
+        roof = {"bound": "tensor", "achieved": tfs, "peak": peaks["bf16_sustained"],
+                "unit": "TFLOP/s", "frac": tfs / peaks["bf16_sustained"]}
+    else:
+        roof = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm"], "unit": "GB/s",
+                "frac": gbs / peaks["hbm"]}
+    roof.update({"traffic": None, "kernel": "pp::doc_pass_tc<128>",
+                 "peak_source": peaks["source"] + (" sustained bf16" if roof["bound"] == "tensor"
+                                                   else " copy"),
+                 "doc_us": durs["doc"] * 1e3, "suffix_merge_us": durs["suffix"] * 1e3,
+                 "doc_hbm_gbs": gbs, "doc_tflops": tfs,
+                 "frac_hbm": gbs / peaks["hbm"], "frac_tensor_burst": tfs / peaks["bf16"],
+                 "frac_tensor_sustained": tfs / peaks["bf16_sustained"]})
+
+    cpu = None
+    if rank == 0 and world == 1 and args.cpu_seconds > 0:
+        cval, threads, desc = oracle_sample(W, args.cpu_seconds)
+        cpu = {"value": cval, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc}
+
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": args.workload, "layers": nl, "H": W.H, "d": W.d,
+                       "doc_tokens": W.N, "streams": W.P,
+                       "suffix_tokens": W.suffix_tokens(),
+                       "l2": "inputs larger than L2 (8.6 GB of document KV per step)"
+                             if nl == 32 else "per-layer document KV exceeds L2",
+                       "parallelism": f"replicas x{world}"},
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+            "gpu_launches": step.kernels_per_step() * args.steps,
+            "roofline": roof,
+            "cpu_baseline": cpu,
+            "clocks": clocks.summary()}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    del step.graph
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

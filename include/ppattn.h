@@ -106,12 +106,18 @@ typedef struct pp_kv_layer {
  *                           returns without hanging.
  *   wait_limit_log2         test only: 0 = default bound on in-kernel waits
  *                           (about 2^31 clock cycles); else 2^value cycles.
+ *   events                  NULL, or 3 caller-created cudaEvent_t handles that
+ *                           decode/prefill record on `stream` before the
+ *                           document pass, after it, and after the suffix
+ *                           pass with its merge (per-kernel timing with CUDA
+ *                           events; the work done is unchanged).
  */
 typedef struct pp_options {
     int32_t splits;
     int32_t ablation_doc_per_stream;
     int32_t debug_inject_timeout;
     int32_t wait_limit_log2;
+    void **events;
 } pp_options;
 
 /* Human-readable name of a pp_status value. */
@@ -140,7 +146,7 @@ pp_status pp_kv_append(const pp_kv_layer *layer, const uint16_t *k, const uint16
 
 /*
  * Workspace bytes pp_decode_attn needs for P query rows (fp32 partial
- * results of the split document pass and of the suffix pass).  The split
+ * results of the split document pass; 0 when doc_len is 0).  The split
  * plan depends on the SM count of the CURRENT device: query with the device
  * that will run the call.  Returns 0 on bad arguments or without a device.
  */
@@ -210,6 +216,14 @@ pp_status pp_debug_visibility(const pp_kv_layer *layer, int32_t doc_len, const i
  */
 pp_status pp_debug_split_plan(int32_t rows, int32_t H, int32_t doc_len, int32_t ctas,
                               int64_t *h_out, int32_t h_out_len);
+
+/*
+ * Test aid: the document pass's two base-2 exponentials on n device floats:
+ * y_poly[i] from the FMA-pipe polynomial (range reduction + degree-3
+ * minimax), y_hw[i] from the hardware ex2 instruction.  No counterpart on
+ * the pages; it exists so tests can bound the polynomial's error.
+ */
+pp_status pp_debug_exp2(const float *x, float *y_poly, float *y_hw, int32_t n, void *stream);
 
 /* Copy the layer's device status word to *h_status (synchronises stream). */
 pp_status pp_get_device_status(const pp_kv_layer *layer, int32_t *h_status, void *stream);

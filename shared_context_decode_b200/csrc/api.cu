@@ -2,7 +2,7 @@
 //
 // Host code here validates arguments, derives the document split plan,
 // carves the caller's workspace and launches the kernels in stream order:
-//   decode / prefill:  [document pass] -> suffix pass -> log-sum-exp merge
+//   decode / prefill:  [document pass] -> suffix pass with the merge fused
 // Nothing here allocates device memory or synchronises (except
 // pp_get_device_status), so the calls can be captured in a CUDA graph.
 #include <algorithm>
@@ -89,17 +89,16 @@ SplitPlan plan_for(int rows, int H, int doc_len, const pp_options* opt) {
 }
 
 struct WsLayout {
-  size_t doc_o, doc_ml, suf_o, suf_ml, total;
+  size_t doc_o, doc_ml, total;
 };
 
-WsLayout ws_layout(int rows, int H, int d, const SplitPlan& p) {
+// Only the document pass leaves partial results in the workspace.
+WsLayout ws_layout(const SplitPlan& p, int d) {
   WsLayout w;
   const size_t slots = (size_t)p.units * p.max_chunks * pp::kGroupRows;
   w.doc_o = 0;
   w.doc_ml = w.doc_o + up(slots * d * sizeof(float));
-  w.suf_o = w.doc_ml + up(slots * 2 * sizeof(float));
-  w.suf_ml = w.suf_o + up((size_t)rows * H * d * sizeof(float));
-  w.total = w.suf_ml + up((size_t)rows * H * 2 * sizeof(float));
+  w.total = w.doc_ml + up(slots * 2 * sizeof(float));
   return w;
 }
 
@@ -108,8 +107,6 @@ Partials carve(void* ws, const WsLayout& w) {
   Partials p;
   p.doc_o = reinterpret_cast<float*>(b + w.doc_o);
   p.doc_ml = reinterpret_cast<float*>(b + w.doc_ml);
-  p.suf_o = reinterpret_cast<float*>(b + w.suf_o);
-  p.suf_ml = reinterpret_cast<float*>(b + w.suf_ml);
   return p;
 }
 
@@ -134,31 +131,37 @@ pp_status attend(const pp_kv_layer* L, int32_t doc_len, const uint16_t* q, const
   const SplitPlan plan = plan_for(rows, L->H, doc_len, opt);
   const bool has_doc = doc_len > 0;
   if (has_doc && plan.C < 1) return PP_ERR_CUDA;  // no device to size the split for
-  const WsLayout w = ws_layout(rows, L->H, L->d, plan);
-  if (!ws || !aligned(ws, kAlign)) return PP_ERR_INVALID_ARG;
+  const WsLayout w = ws_layout(plan, L->d);
+  if (w.total > 0 && (!ws || !aligned(ws, kAlign))) return PP_ERR_INVALID_ARG;
   if (ws_bytes < w.total) return PP_ERR_CAPACITY;
+  const int sms = sm_count();
+  if (sms < 1) return PP_ERR_CUDA;
   const Partials part = carve(ws, w);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaEvent_t* ev = (opt && opt->events) ? reinterpret_cast<cudaEvent_t*>(opt->events) : nullptr;
+  auto mark = [&](int i) { return ev ? cudaEventRecord(ev[i], st) : cudaSuccess; };
+  if (mark(0) != cudaSuccess) return PP_ERR_CUDA;
   if (has_doc) {
     cudaError_t e;
     if (opt && opt->ablation_doc_per_stream)
-      e = pp::launch_doc_per_stream(*L, doc_len, q, q_sid, rows, scale, plan.max_chunks, part, st);
+      e = pp::launch_doc_per_stream(*L, doc_len, q, rows, scale, plan.max_chunks, part, st);
     else
       e = pp::launch_doc_pass_tc(*L, doc_len, q, rows, scale, plan, part, wait_limit(opt),
                                  opt ? opt->debug_inject_timeout : 0, st);
     if (e != cudaSuccess) return PP_ERR_CUDA;
   }
-  if ((s = from_cuda(pp::launch_suffix_pass(*L, q, q_sid, q_pos, rows, scale, part, st))) != PP_OK)
+  if (mark(1) != cudaSuccess) return PP_ERR_CUDA;
+  if ((s = from_cuda(pp::launch_suffix_merge(*L, q, q_sid, q_pos, rows, scale, plan, has_doc, part,
+                                             o, lse, wait_limit(opt), sms, st))) != PP_OK)
     return s;
-  return from_cuda(pp::launch_lse_merge(rows, L->H, L->d, L->P_max, plan, has_doc, q_sid, part, o,
-                                        lse, st));
+  return from_cuda(mark(2));
 }
 
 size_t workspace(int32_t rows, int32_t H, int32_t d, int32_t doc_len, const pp_options* opt) {
   if (rows < 0 || H < 1 || (d != 64 && d != 128) || doc_len < 0) return 0;
   const SplitPlan plan = plan_for(rows, H, doc_len, opt);
   if (doc_len > 0 && plan.C < 1) return 0;
-  return ws_layout(rows, H, d, plan).total;
+  return ws_layout(plan, d).total;
 }
 
 }  // namespace
@@ -252,6 +255,15 @@ PP_API pp_status pp_debug_split_plan(int32_t rows, int32_t H, int32_t doc_len, i
     h_out[6 + 2 * u] = p.W ? pp::plan_cta_of(p, (int64_t)u * p.T + p.T - 1) : -1;
   }
   return PP_OK;
+}
+
+PP_API pp_status pp_debug_exp2(const float* x, float* y_poly, float* y_hw, int32_t n,
+                               void* stream) {
+  if (n < 0) return PP_ERR_INVALID_ARG;
+  if (n == 0) return PP_OK;
+  if (!x || !y_poly || !y_hw || !aligned(x, 4) || !aligned(y_poly, 4) || !aligned(y_hw, 4))
+    return PP_ERR_INVALID_ARG;
+  return from_cuda(pp::launch_exp2(x, y_poly, y_hw, n, static_cast<cudaStream_t>(stream)));
 }
 
 PP_API pp_status pp_get_device_status(const pp_kv_layer* layer, int32_t* h_status, void* stream) {

@@ -58,6 +58,77 @@ __device__ __forceinline__ uint32_t f2_to_bf2(float a, float b) {
 }
 
 // ---------------------------------------------------------------------------
+// Blackwell fp32 arithmetic: 3-input max and packed (f32x2) add / fma.
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  uint64_t ra, rb, rc, rd;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(ra) : "f"(a.x), "f"(a.y));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(rb) : "f"(b.x), "f"(b.y));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(rc) : "f"(c.x), "f"(c.y));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(rd) : "l"(ra), "l"(rb), "l"(rc));
+  float2 d;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(d.x), "=f"(d.y) : "l"(rd));
+  return d;
+}
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+  uint64_t ra, rb, rd;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(ra) : "f"(a.x), "f"(a.y));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(rb) : "f"(b.x), "f"(b.y));
+  asm("add.f32x2 %0, %1, %2;" : "=l"(rd) : "l"(ra), "l"(rb));
+  float2 d;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(d.x), "=f"(d.y) : "l"(rd));
+  return d;
+}
+// a + b rounded toward -infinity, both lanes.
+__device__ __forceinline__ float2 fadd2_rm(float2 a, float2 b) {
+  uint64_t ra, rb, rd;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(ra) : "f"(a.x), "f"(a.y));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(rb) : "f"(b.x), "f"(b.y));
+  asm("add.rm.f32x2 %0, %1, %2;" : "=l"(rd) : "l"(ra), "l"(rb));
+  float2 d;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(d.x), "=f"(d.y) : "l"(rd));
+  return d;
+}
+
+// Hardware base-2 exponential (MUFU), flush-to-zero.
+__device__ __forceinline__ float ex2_mufu(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// 2^x on the FMA pipe, for two values at once, so part of the softmax's
+// exponentials can bypass the MUFU unit.  Range reduction: x = n + f with
+// n = floor(x) (x + 1.5*2^23 rounded toward -inf leaves n in the low mantissa
+// bits) and f in [0, 1); 2^f from a degree-3 polynomial fitted for minimum
+// maximum relative error on [0, 1) with Lawson's iteratively reweighted least
+// squares (max relative error 8.4e-5, far below the 2^-8 step of the bf16
+// probabilities it feeds); then n is added to the exponent field.  x is
+// clamped at -126 (2^f can be just below 1, exponent field 126, so n >= -126
+// keeps the field >= 0): -inf and underflow give at most 2^-125, zero for
+// every use here.  Valid for x <= 64.
+__device__ __forceinline__ float2 ex2_poly2(float2 x) {
+  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+  x.x = fmaxf(x.x, -126.f);
+  x.y = fmaxf(x.y, -126.f);
+  const float2 t = fadd2_rm(x, make_float2(kMagic, kMagic));
+  const float2 n = fadd2(t, make_float2(-kMagic, -kMagic));
+  const float2 f = fadd2(x, make_float2(-n.x, -n.y));
+  float2 p = ffma2(make_float2(0.07808296f, 0.07808296f), f, make_float2(0.22612518f, 0.22612518f));
+  p = ffma2(p, f, make_float2(0.69573334f, 0.69573334f));
+  p = ffma2(p, f, make_float2(0.99994152f, 0.99994152f));
+  // (t_bits << 23) equals n << 23 modulo 2^32: the magic constant's low 9 bits are zero.
+  float2 r;
+  r.x = __int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23));
+  r.y = __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23));
+  return r;
+}
+
+// ---------------------------------------------------------------------------
 // Split plan of the document pass.  Work is the linear range of
 // units * T tiles, unit u = group * H + head, T = ceil(doc_len / kBN).  CTA c
 // owns tiles [floor(c*W/C), floor((c+1)*W/C)); every (unit, CTA) overlap is a
@@ -80,12 +151,11 @@ __host__ __device__ __forceinline__ int32_t plan_cta_of(const SplitPlan& p, int6
 }
 
 // ---------------------------------------------------------------------------
-// Workspace layout shared by the document pass, the suffix pass and the merge.
+// Workspace: the document pass's partial results, read by the merge in the
+// suffix kernel's epilogue.
 struct Partials {
   float* doc_o;     // [units*max_chunks][kGroupRows][d]  un-normalised
   float* doc_ml;    // [units*max_chunks][kGroupRows][2]  (max, sum), log2 domain
-  float* suf_o;     // [rows][H][d]
-  float* suf_ml;    // [rows][H][2]
 };
 
 // ---------------------------------------------------------------------------
@@ -159,8 +229,30 @@ __device__ __forceinline__ void tma_load_3d(void* smem_dst, const void* tmap, ui
       : "memory");
 }
 
+// 1-D bulk copy global -> shared (TMA engine, no tensor map, no multicast).
+// Both addresses 16-byte aligned, size a multiple of 16 bytes.
+__device__ __forceinline__ void bulk_load(void* smem_dst, const void* gmem_src, uint32_t bytes,
+                                          uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(gmem_src)), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
 __device__ __forceinline__ void prefetch_tmap(const void* tmap) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
+}
+
+// One lane of a converged warp (elect.sync).  Issue code that a single thread
+// must run (MMA, commit, TMA) is executed by the whole warp with only the
+// elected lane issuing, so every operand stays warp-uniform: a loop run by a
+// lone lane measured about 3x slower per MMA on B200.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile("{\n\t.reg .pred P;\n\telect.sync _|P, 0xffffffff;\n\tselp.u32 %0, 1, 0, P;\n\t}"
+               : "=r"(pred));
+  return pred != 0;
 }
 
 // tcgen05 (5th-generation tensor core) ----------------------------------------
@@ -235,6 +327,15 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
       "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
       "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
       "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15])
       : "memory");
 }
 __device__ __forceinline__ void tmem_ld_wait() {

@@ -41,7 +41,7 @@ namespace pp {
 // Register split: the block is launched with kRegsLaunch registers per thread
 // (384 * 168 = 64512); warps 0-3 drop to kRegsLow and the 8 softmax warps
 // rise to kRegsHigh, which adds up to exactly the launch total.
-constexpr int kRegsLaunch = 168, kRegsLow = 56, kRegsHigh = 224;
+constexpr int kRegsLaunch = 168, kRegsLow = 88, kRegsHigh = 208;
 static_assert(128 * kRegsLow + 256 * kRegsHigh <= 384 * kRegsLaunch, "register split");
 
 struct DocTcParams {
@@ -137,11 +137,10 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
-__device__ __forceinline__ float ex2(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
+// Softmax exponentials: pairs p with p % 5 in {1, 3} go to the FMA-pipe
+// polynomial, the rest to MUFU, balancing the two pipes (MUFU issues a warp's
+// 32 lanes in 8 cycles; the polynomial costs about 5 issue slots a value).
+__device__ __forceinline__ constexpr bool use_poly(int pair) { return pair % 5 == 1 || pair % 5 == 3; }
 
 template <int D>
 __global__ void __launch_bounds__(384, 1)
@@ -211,159 +210,190 @@ __global__ void __launch_bounds__(384, 1)
 
   if (warp == 0) {
     // ------------------------------------------------ Q and K producer ----
+    // The whole warp walks the schedule; the elected lane issues the copies.
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLow));
-    if (lane == 0) {
-      int64_t t = t_begin;
-      Seg s;
-      int kt = 0, nseg = 0;
-      bool ok = true;
-      while (ok && next_seg(p, t, t_end, cta, s)) {
-        if (nseg > 0 && !(ok = mbar_wait(B.q_empty, (nseg - 1) & 1, abort_flag, p.wait_limit, p.status)))
-          break;
+    int64_t t = t_begin;
+    Seg s;
+    int kt = 0, nseg = 0;
+    bool ok = true;
+    while (ok && next_seg(p, t, t_end, cta, s)) {
+      if (nseg > 0 &&
+          !(ok = warp_wait(B.q_empty, (nseg - 1) & 1, abort_flag, p.wait_limit, p.status)))
+        break;
+      if (elect_one()) {
         mbar_arrive_expect_tx(B.q_full, s.nm * C::KH * C::BOX);
         for (int mt = 0; mt < s.nm; ++mt)
           for (int kh = 0; kh < C::KH; ++kh)
             tma_load_3d(smem + C::OFF_Q + (mt * C::KH + kh) * C::BOX, &tmQ, B.q_full, kh * 64, s.h,
                         s.g * kGroupRows + mt * 128);
-        for (int j = s.j0; j < s.j1; ++j, ++kt) {
-          const int st = kt % C::NK, f = kt / C::NK;
-          if (f > 0 && !(ok = mbar_wait(B.k_empty + st, (f - 1) & 1, abort_flag, p.wait_limit, p.status)))
-            break;
-          mbar_arrive_expect_tx(B.k_full + st, C::KH * C::BOX);
-          if (p.inject_timeout && kt == 0) continue;  // test hook: this copy never lands
-          for (int kh = 0; kh < C::KH; ++kh)
-            tma_load_3d(smem + C::OFF_K + st * C::KV_STAGE + kh * C::BOX, &tmK, B.k_full + st,
-                        kh * 64, j * kBN, s.h);
-        }
-        ++nseg;
       }
-      if (!ok) {
-        // Drain: wait (bounded, abort flag ignored) for the copies still in flight.
-        for (int back = 1; back <= C::NK && kt - back >= 0; ++back) {
-          const int k2 = kt - back;
-          if (p.inject_timeout && k2 == 0) continue;
-          volatile int never = 0;
-          mbar_wait(B.k_full + k2 % C::NK, (k2 / C::NK) & 1, &never, p.wait_limit, nullptr);
+      for (int j = s.j0; j < s.j1; ++j, ++kt) {
+        const int st = kt % C::NK, f = kt / C::NK;
+        if (f > 0 &&
+            !(ok = warp_wait(B.k_empty + st, (f - 1) & 1, abort_flag, p.wait_limit, p.status)))
+          break;
+        if (elect_one()) {
+          mbar_arrive_expect_tx(B.k_full + st, C::KH * C::BOX);
+          if (!(p.inject_timeout && kt == 0))  // test hook: this copy never lands
+            for (int kh = 0; kh < C::KH; ++kh)
+              tma_load_3d(smem + C::OFF_K + st * C::KV_STAGE + kh * C::BOX, &tmK, B.k_full + st,
+                          kh * 64, j * kBN, s.h);
         }
+      }
+      ++nseg;
+    }
+    if (!ok && lane == 0) {
+      // Drain: wait (bounded, abort flag ignored) for the copies still in flight.
+      for (int back = 1; back <= C::NK && kt - back >= 0; ++back) {
+        const int k2 = kt - back;
+        if (p.inject_timeout && k2 == 0) continue;
+        volatile int never = 0;
+        mbar_wait(B.k_full + k2 % C::NK, (k2 / C::NK) & 1, &never, p.wait_limit, nullptr);
       }
     }
   } else if (warp == 3) {
     // -------------------------------------------------------- V producer ----
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLow));
-    if (lane == 0) {
-      int64_t t = t_begin;
-      Seg s;
-      int vt = 0;
-      bool ok = true;
-      while (ok && next_seg(p, t, t_end, cta, s)) {
-        for (int j = s.j0; j < s.j1; ++j, ++vt) {
-          const int st = vt % C::NV, f = vt / C::NV;
-          if (f > 0 && !(ok = mbar_wait(B.v_empty + st, (f - 1) & 1, abort_flag, p.wait_limit, p.status)))
-            break;
+    int64_t t = t_begin;
+    Seg s;
+    int vt = 0;
+    bool ok = true;
+    while (ok && next_seg(p, t, t_end, cta, s)) {
+      for (int j = s.j0; j < s.j1; ++j, ++vt) {
+        const int st = vt % C::NV, f = vt / C::NV;
+        if (f > 0 &&
+            !(ok = warp_wait(B.v_empty + st, (f - 1) & 1, abort_flag, p.wait_limit, p.status)))
+          break;
+        if (elect_one()) {
           mbar_arrive_expect_tx(B.v_full + st, C::KH * C::BOX);
           for (int kh = 0; kh < C::KH; ++kh)
             tma_load_3d(smem + C::OFF_V + st * C::KV_STAGE + kh * C::BOX, &tmV, B.v_full + st,
                         kh * 64, j * kBN, s.h);
         }
       }
-      if (!ok) {
-        for (int back = 1; back <= C::NV && vt - back >= 0; ++back) {
-          const int v2 = vt - back;
-          volatile int never = 0;
-          mbar_wait(B.v_full + v2 % C::NV, (v2 / C::NV) & 1, &never, p.wait_limit, nullptr);
-        }
+    }
+    if (!ok && lane == 0) {
+      for (int back = 1; back <= C::NV && vt - back >= 0; ++back) {
+        const int v2 = vt - back;
+        volatile int never = 0;
+        mbar_wait(B.v_full + v2 % C::NV, (v2 / C::NV) & 1, &never, p.wait_limit, nullptr);
       }
     }
   } else if (warp == 1) {
     // --------------------------------------------------------- MMA issuer ----
+    // All 32 lanes run this loop (operands stay warp-uniform); elect_one()
+    // issues each MMA and commit.  k-loops are unrolled with constant
+    // descriptor offsets.
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLow));
-    if (lane == 0) {
-      constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, kBN, 0);
-      constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, D, 1);
-      const uint32_t sQ = smem_u32(smem + C::OFF_Q);
-      const uint32_t sK = smem_u32(smem + C::OFF_K);
-      const uint32_t sV = smem_u32(smem + C::OFF_V);
-      auto issue_qk = [&](int mt, int kslot) {
-        const uint32_t d_t = tmem + (mt ? C::T_S1 : C::T_S0);
+    constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, kBN, 0);
+    constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, D, 1);
+    // Descriptors advance by adding (byte offset >> 4) to the start-address
+    // field; every tile stays inside shared memory, so no carry leaves it.
+    const uint64_t dQ = smem_desc_sw128(smem_u32(smem + C::OFF_Q), 16, 1024);
+    const uint64_t dK = smem_desc_sw128(smem_u32(smem + C::OFF_K), 16, 1024);
+    const uint64_t dV = smem_desc_sw128(smem_u32(smem + C::OFF_V), C::BOX, 1024);
+    auto issue_qk = [&](int mt, int kslot) {
+      const uint32_t d_t = tmem + (mt ? C::T_S1 : C::T_S0);
+      const uint64_t a0 = dQ + (uint64_t)((mt * C::KH * C::BOX) >> 4);
+      const uint64_t b0 = dK + (uint64_t)((kslot * C::KV_STAGE) >> 4);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (uint32_t)((kk >> 2) * C::BOX + (kk & 3) * 32);
-          const uint64_t a = smem_desc_sw128(sQ + mt * C::KH * C::BOX + off, 16, 1024);
-          const uint64_t b = smem_desc_sw128(sK + kslot * C::KV_STAGE + off, 16, 1024);
-          mma_ss(d_t, a, b, IDESC_QK, kk > 0 ? 1u : 0u);
-        }
-      };
-      auto issue_pv = [&](int mt, int vslot, bool acc) {
-        const uint32_t d_t = tmem + (mt ? C::T_O1 : C::T_O0);
-        const uint32_t a_t = tmem + (mt ? C::T_S1 : C::T_S0);
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint64_t off = (uint64_t)(((kk >> 2) * C::BOX + (kk & 3) * 32) >> 4);
+        if (elect_one()) mma_ss(d_t, a0 + off, b0 + off, IDESC_QK, kk > 0 ? 1u : 0u);
+      }
+    };
+    auto issue_pv = [&](int mt, int vslot, bool acc) {
+      const uint32_t d_t = tmem + (mt ? C::T_O1 : C::T_O0);
+      const uint32_t a_t = tmem + (mt ? C::T_S1 : C::T_S0);
+      const uint64_t b0 = dV + (uint64_t)((vslot * C::KV_STAGE) >> 4);
 #pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk) {
-          const uint64_t b = smem_desc_sw128(sV + vslot * C::KV_STAGE + kk * 16 * 128, C::BOX, 1024);
-          mma_ts(d_t, a_t + kk * 8, b, IDESC_PV, (acc || kk > 0) ? 1u : 0u);
-        }
-      };
-      int64_t t = t_begin;
-      Seg s;
-      int kt = 0, vt = 0, nseg = 0;
-      uint32_t pf_ph[2] = {0, 0};
-      bool ok = true;
-      while (ok && next_seg(p, t, t_end, cta, s)) {
-        if (!(ok = mbar_wait(B.q_full, nseg & 1, abort_flag, p.wait_limit, p.status))) break;
-        tc_fence_after();
-        if (!(ok = mbar_wait(B.k_full + kt % C::NK, (kt / C::NK) & 1, abort_flag, p.wait_limit, p.status)))
+      for (int kk = 0; kk < kBN / 16; ++kk)
+        if (elect_one())
+          mma_ts(d_t, a_t + kk * 8, b0 + (uint64_t)((kk * 16 * 128) >> 4), IDESC_PV,
+                 (acc || kk > 0) ? 1u : 0u);
+    };
+    auto commit = [&](uint64_t* bar_) {
+      if (elect_one()) tc_commit(bar_);
+      __syncwarp();
+    };
+    int64_t t = t_begin;
+    Seg s;
+    int kt = 0, vt = 0, nseg = 0;
+    uint32_t pf_ph0 = 0, pf_ph1 = 0;
+    int used0 = 0, used1 = 0;  // segments in which each M tile has been active
+    bool ok = true;
+    while (ok && next_seg(p, t, t_end, cta, s)) {
+      if (!(ok = warp_wait(B.q_full, nseg & 1, abort_flag, p.wait_limit, p.status))) break;
+      if (!(ok = warp_wait(B.k_full + kt % C::NK, (kt / C::NK) & 1, abort_flag, p.wait_limit,
+                           p.status)))
+        break;
+      tc_fence_after();
+      issue_qk(0, kt % C::NK);
+      commit(B.s_full + 0);
+      if (s.nm > 1) {
+        issue_qk(1, kt % C::NK);
+        commit(B.s_full + 1);
+      }
+      commit(B.k_empty + kt % C::NK);
+      ++kt;
+      if (s.j1 - s.j0 == 1) commit(B.q_empty);
+      for (int j = s.j0; ok && j < s.j1; ++j) {
+        const int vslot = vt % C::NV;
+        if (!(ok = warp_wait(B.v_full + vslot, (vt / C::NV) & 1, abort_flag, p.wait_limit, p.status)))
           break;
+        const bool has_next = j + 1 < s.j1;
+        const int kslot = kt % C::NK;
+        // ---- M tile 0
+        // The first O += P V of a segment overwrites O: wait until the
+        // softmax has read out the previous segment that used this tile.
+        if (j == s.j0 && used0 > 0 &&
+            !(ok = warp_wait(B.o_free + 0, (used0 - 1) & 1, abort_flag, p.wait_limit, p.status)))
+          break;
+        if (!(ok = warp_wait(B.p_full + 0, pf_ph0, abort_flag, p.wait_limit, p.status))) break;
+        pf_ph0 ^= 1;
         tc_fence_after();
-        for (int mt = 0; mt < s.nm; ++mt) {
-          issue_qk(mt, kt % C::NK);
-          tc_commit(B.s_full + mt);
-        }
-        tc_commit(B.k_empty + kt % C::NK);
-        ++kt;
-        if (s.j1 - s.j0 == 1) tc_commit(B.q_empty);
-        for (int j = s.j0; ok && j < s.j1; ++j) {
-          const int vslot = vt % C::NV;
-          if (!(ok = mbar_wait(B.v_full + vslot, (vt / C::NV) & 1, abort_flag, p.wait_limit, p.status)))
+        issue_pv(0, vslot, j > s.j0);
+        if (has_next) {
+          if (!(ok = warp_wait(B.k_full + kslot, (kt / C::NK) & 1, abort_flag, p.wait_limit,
+                               p.status)))
             break;
           tc_fence_after();
-          const bool has_next = j + 1 < s.j1;
-          const int kslot = kt % C::NK;
-          if (j == s.j0 && nseg > 0) {
-            for (int mt = 0; mt < 2 && ok; ++mt)
-              ok = mbar_wait(B.o_free + mt, (nseg - 1) & 1, abort_flag, p.wait_limit, p.status);
-            if (!ok) break;
-            tc_fence_after();
-          }
-          for (int mt = 0; mt < s.nm; ++mt) {
-            if (!(ok = mbar_wait(B.p_full + mt, pf_ph[mt], abort_flag, p.wait_limit, p.status))) break;
-            pf_ph[mt] ^= 1;
-            tc_fence_after();
-            issue_pv(mt, vslot, j > s.j0);
-            if (has_next) {
-              if (mt == 0) {
-                if (!(ok = mbar_wait(B.k_full + kslot, (kt / C::NK) & 1, abort_flag, p.wait_limit,
-                                     p.status)))
-                  break;
-                tc_fence_after();
-              }
-              issue_qk(mt, kslot);
-              tc_commit(B.s_full + mt);
-            } else {
-              tc_commit(B.o_done + mt);
-            }
-          }
-          if (!ok) break;
-          tc_commit(B.v_empty + vslot);
-          ++vt;
+          issue_qk(0, kslot);
+          commit(B.s_full + 0);
+        } else {
+          commit(B.o_done + 0);
+        }
+        // ---- M tile 1
+        if (s.nm > 1) {
+          if (j == s.j0 && used1 > 0 &&
+              !(ok = warp_wait(B.o_free + 1, (used1 - 1) & 1, abort_flag, p.wait_limit, p.status)))
+            break;
+          if (!(ok = warp_wait(B.p_full + 1, pf_ph1, abort_flag, p.wait_limit, p.status))) break;
+          pf_ph1 ^= 1;
+          tc_fence_after();
+          issue_pv(1, vslot, j > s.j0);
           if (has_next) {
-            tc_commit(B.k_empty + kslot);
-            ++kt;
-            if (j + 2 == s.j1) tc_commit(B.q_empty);
+            issue_qk(1, kslot);
+            commit(B.s_full + 1);
+          } else {
+            commit(B.o_done + 1);
           }
         }
-        ++nseg;
+        commit(B.v_empty + vslot);
+        ++vt;
+        if (has_next) {
+          commit(B.k_empty + kslot);
+          ++kt;
+          if (j + 2 == s.j1) commit(B.q_empty);
+        }
       }
-      if (!ok) {
-        tc_commit(B.drain);
+      ++used0;
+      if (s.nm > 1) ++used1;
+      ++nseg;
+    }
+    if (!ok) {
+      commit(B.drain);
+      if (lane == 0) {
         volatile int never = 0;
         mbar_wait(B.drain, 0, &never, p.wait_limit, nullptr);
       }
@@ -382,7 +412,6 @@ __global__ void __launch_bounds__(384, 1)
     int64_t t = t_begin;
     Seg s;
     uint32_t s_ph = 0, od_ph = 0;
-    int nseg = 0;
     bool ok = true;
     while (ok && next_seg(p, t, t_end, cta, s)) {
       if (wg < s.nm) {
@@ -403,17 +432,56 @@ __global__ void __launch_bounds__(384, 1)
               for (int e = 0; e < 32; ++e)
                 if (c * 32 + e >= kvalid) r[c][e] = __float_as_uint(-INFINITY);
           }
-          float mx = -INFINITY;
+          // row maximum: 8 independent chains of 3-input max
+          float mc[8];
 #pragma unroll
-          for (int c = 0; c < 4; ++c)
+          for (int k = 0; k < 8; ++k) mc[k] = -INFINITY;
 #pragma unroll
-            for (int e = 0; e < 32; ++e) mx = fmaxf(mx, __uint_as_float(r[c][e]));
+          for (int i = 0; i < 128; i += 2)
+            mc[(i >> 1) & 7] = fmax3(mc[(i >> 1) & 7], __uint_as_float(r[i >> 5][i & 31]),
+                                     __uint_as_float(r[i >> 5][(i & 31) + 1]));
+          const float mx = fmax3(fmax3(mc[0], mc[1], mc[2]), fmax3(mc[3], mc[4], mc[5]),
+                                 fmaxf(mc[6], mc[7]));
           const float m_new = fmaxf(m, mx * p.sl2);
           // Lazy rescale: keep a stale maximum unless the new one exceeds it
           // by more than 2^8 (probabilities then stay below 256).
           const bool need = m_new > m + 8.f;
+          const float m_old = m;
+          if (need) {
+            l *= ex2_mufu(m - m_new);
+            m = m_new;
+          }
+          // P = 2^(S * scale*log2e - m) as bf16 pairs, written over S's first
+          // 64 columns chunk by chunk; row sum in 4 packed partial sums.
+          const float2 sl2v = make_float2(p.sl2, p.sl2), negm = make_float2(-m, -m);
+          float2 rs[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int e = 0; e < 32; e += 2) {
+              const int pr_i = c * 16 + (e >> 1);
+              const float2 a = ffma2(make_float2(__uint_as_float(r[c][e]), __uint_as_float(r[c][e + 1])),
+                                     sl2v, negm);
+              float2 pv;
+              if (use_poly(pr_i)) {
+                pv = ex2_poly2(a);
+              } else {
+                pv.x = ex2_mufu(a.x);
+                pv.y = ex2_mufu(a.y);
+              }
+              rs[pr_i & 1] = fadd2(rs[pr_i & 1], pv);
+              pk[e >> 1] = f2_to_bf2(pv.x, pv.y);
+            }
+            tmem_st16(t_S + c * 16, pk);
+          }
+          l += (rs[0].x + rs[0].y) + (rs[1].x + rs[1].y);
+          // O rescale for rows whose maximum moved (rare; S is dead by now).
+          // O is stable here: O += P V of the previous tile has completed
+          // (committed before this tile's S) and this tile's is not issued
+          // before p_full.
           if (j > s.j0 && __any_sync(0xffffffffu, need)) {
-            const float f = need ? ex2(m - m_new) : 1.f;
+            const float f = need ? ex2_mufu(m_old - m) : 1.f;
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) {
               uint32_t o[32];
@@ -423,26 +491,7 @@ __global__ void __launch_bounds__(384, 1)
               for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
               tmem_st32(t_O + c * 32, o);
             }
-            tmem_st_wait();
           }
-          if (need) {
-            l *= ex2(m - m_new);
-            m = m_new;
-          }
-          float rs = 0.f;
-          uint32_t pk[2][32];
-#pragma unroll
-          for (int c = 0; c < 4; ++c)
-#pragma unroll
-            for (int e = 0; e < 32; e += 2) {
-              const float p0 = ex2(fmaf(__uint_as_float(r[c][e]), p.sl2, -m));
-              const float p1 = ex2(fmaf(__uint_as_float(r[c][e + 1]), p.sl2, -m));
-              rs += p0 + p1;
-              pk[c >> 1][(c & 1) * 16 + (e >> 1)] = f2_to_bf2(p0, p1);
-            }
-          l += rs;
-          tmem_st32(t_S, pk[0]);
-          tmem_st32(t_S + 32, pk[1]);
           tmem_st_wait();
           tc_fence_before();
           mbar_arrive(B.p_full + wg);
@@ -470,10 +519,9 @@ __global__ void __launch_bounds__(384, 1)
           }
         }
         if (valid) reinterpret_cast<float2*>(p.doc_ml)[prow] = make_float2(m, l);
+        tc_fence_before();
+        mbar_arrive(B.o_free + wg);
       }
-      tc_fence_before();
-      mbar_arrive(B.o_free + wg);
-      ++nseg;
     }
   }
 

@@ -19,17 +19,18 @@ cudaError_t launch_kv_reset(const pp_kv_layer& L, cudaStream_t st);
 cudaError_t launch_doc_pass_tc(const pp_kv_layer& L, int doc_len, const uint16_t* q, int rows,
                                float scale, const SplitPlan& plan, const Partials& part,
                                long long wait_limit, int inject_timeout, cudaStream_t st);
-cudaError_t launch_doc_per_stream(const pp_kv_layer& L, int doc_len, const uint16_t* q,
-                                  const int16_t* q_sid, int rows, float scale, int max_chunks,
-                                  const Partials& part, cudaStream_t st);
-cudaError_t launch_suffix_pass(const pp_kv_layer& L, const uint16_t* q, const int16_t* q_sid,
-                               const int32_t* q_pos, int rows, float scale, const Partials& part,
-                               cudaStream_t st);
-cudaError_t launch_lse_merge(int rows, int H, int d, int P_max, const SplitPlan& plan, bool has_doc,
-                             const int16_t* q_sid, const Partials& part, uint16_t* o, float* lse,
-                             cudaStream_t st);
+cudaError_t launch_doc_per_stream(const pp_kv_layer& L, int doc_len, const uint16_t* q, int rows,
+                                  float scale, int max_chunks, const Partials& part,
+                                  cudaStream_t st);
+// Suffix pass with the log-sum-exp merge in its epilogue; writes o and lse.
+cudaError_t launch_suffix_merge(const pp_kv_layer& L, const uint16_t* q, const int16_t* q_sid,
+                                const int32_t* q_pos, int rows, float scale, const SplitPlan& plan,
+                                bool has_doc, const Partials& part, uint16_t* o, float* lse,
+                                long long wait_limit, int num_sms, cudaStream_t st);
 cudaError_t launch_visibility(const pp_kv_layer& L, int doc_len, const int16_t* q_sid,
                               const int32_t* q_pos, int nq, int32_t* count_out, uint8_t* mask_out,
                               cudaStream_t st);
+
+cudaError_t launch_exp2(const float* x, float* y_poly, float* y_hw, int n, cudaStream_t st);
 
 }  // namespace pp

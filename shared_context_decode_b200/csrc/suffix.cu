@@ -1,73 +1,272 @@
-// K3 / K5: the suffix pass.  One warp per (query row, head) walks the query's
-// own stream segment and applies the stream mask ("Read Once, Answer Many"
-// project page, section "How it works", item 1): a slot counts iff it carries
-// the query's stream id and a position not later than the query's.  The
-// decode step (one row per stream) and the question prefill (rows causal
-// within their question) run the same kernel.
+// K3 + K4: the suffix pass with the log-sum-exp merge fused into its epilogue.
 //
-// Memory layout read: segment (s-1, h) is S_cap contiguous rows of d bf16, so
-// a warp streams one contiguous block.  d/8 lanes share a key (one 16-byte
-// load each); a warp covers 32/(d/8) keys per load and keeps U loads of K and
-// V in flight before using them.  Scores are reduced with warp shuffles.
-// Output: an un-normalised partial (O, max, sum) in the log2 domain, merged
-// with the document partials by the merge kernel.
+// Each query row attends, besides the document, to the slots of its own
+// stream segment that the stream mask admits ("Read Once, Answer Many"
+// project page, section "How it works", item 1: same stream id and not later
+// than the query).  The decode step (one row per stream) and the question
+// prefill (rows causal within their question) run the same kernel.
+//
+// Work item = (query row, head).  Segment (s-1, h) is S_cap contiguous rows of
+// d bf16 ([P_max][H][S_cap][d]), so an item's keys stream as one contiguous
+// block.  Every warp owns a ring of NS shared-memory stages; lane 0 fills them
+// with 1-D TMA bulk copies (CK keys of K and of V per stage) running NS-1
+// chunks ahead of the warp, across item boundaries, so HBM reads overlap the
+// arithmetic without holding the data in registers.  d/8 lanes share a key
+// (16 bytes each), scores are reduced with warp shuffles, softmax is online in
+// the log2 domain.
+//
+// Epilogue (merge): the item's suffix partial is combined with the document
+// pass's partials of the same (row, head):
+//   M = max m_i,  Lsum = sum l_i 2^(m_i - M),  o = sum O_i 2^(m_i - M) / Lsum,
+//   lse = (M + log2 Lsum) ln 2,
+// the softmax over the union of the key sets in max-shifted form.  Rows that
+// are not answer-stream queries, and rows that see nothing, get o = 0 and
+// lse = -inf.
+#include <atomic>
+
 #include "common.cuh"
 #include "internal.h"
 
 namespace pp {
 
 template <int D>
-__device__ __forceinline__ void segment_partial(const pp_kv_layer& L, const uint16_t* __restrict__ q,
-                                                int r, int h, int q_sid, int q_pos, float sl2,
-                                                float* __restrict__ out_o,
-                                                float* __restrict__ out_ml, int lane) {
-  constexpr int LPK = D / 8;    // lanes per key
-  constexpr int KPI = 32 / LPK; // keys per warp-wide load
-  constexpr int U = 4;          // loads in flight per lane (K and V each)
-  const int g = lane / LPK, j = lane % LPK;
+struct SufCfg {
+  static constexpr int LPK = D / 8;        // lanes per key (16 bytes each)
+  static constexpr int KPI = 32 / LPK;     // keys a warp covers per step
+  static constexpr int CK = 16;            // keys per chunk
+  static constexpr int ROW = D * 2;        // bytes per key row
+  static constexpr int HALF = CK * ROW;    // K (or V) part of a stage
+  static constexpr int STAGE = 2 * HALF;
+  static constexpr int NS = 3;             // stages per warp (NS-1 chunks in flight)
+  static constexpr int WARPS = 8;          // warps per CTA
+  static constexpr int TBL = 256;          // item-table entries per warp and round
+  static constexpr int PRE = 4;            // document partials prefetched per key group
+  static constexpr int SMEM = WARPS * NS * STAGE + WARPS * TBL * 16 + 128;
+  static_assert(CK % KPI == 0, "chunk covers whole warp steps");
+};
 
-  const uint4 qv = reinterpret_cast<const uint4*>(q + ((int64_t)r * L.H + h) * D)[j];
-  float qf[8];
-  {
-    const uint32_t w[4] = {qv.x, qv.y, qv.z, qv.w};
+struct SufParams {
+  int rows, H, P_max, S_cap;
+  const uint16_t* q;
+  const int16_t* q_sid;
+  const int32_t* q_pos;
+  const uint16_t* k_suf;
+  const uint16_t* v_suf;
+  const int16_t* sid;
+  const int32_t* pos;
+  const int32_t* len;
+  int32_t* status;
+  float sl2;
+  SplitPlan plan;
+  int has_doc;
+  const float* doc_o;
+  const float* doc_ml;
+  uint16_t* o;
+  float* lse;
+  long long wait_limit;
+};
+
+// Per-item record of the warp's table: stream id (0 when the row is not an
+// answer-stream query), query position, visible-segment length.
+struct ItemRec {
+  int s, qp, n, pad;
+};
+
+// Online-softmax state fold: (m, l, a) <- (m, l, a) (+) (m2, l2, a2).
+__device__ __forceinline__ void fold(float& m, float& l, float (&a)[8], float m2, float l2,
+                                     const float (&a2)[8]) {
+  const float mm = fmaxf(m, m2);
+  const float x = (m == -INFINITY) ? 0.f : exp2f(m - mm);
+  const float y = (m2 == -INFINITY) ? 0.f : exp2f(m2 - mm);
+  l = l * x + l2 * y;
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      const float2 f = bf2_to_f2(w[c]);
-      qf[2 * c] = f.x * sl2;
-      qf[2 * c + 1] = f.y * sl2;
-    }
+  for (int c = 0; c < 8; ++c) a[c] = a[c] * x + a2[c] * y;
+  m = mm;
+}
+
+// Combine the per-key-group states across the warp (xor over the group bits).
+template <int LPK>
+__device__ __forceinline__ void combine_groups(float& m, float& l, float (&a)[8]) {
+#pragma unroll
+  for (int o = LPK; o < 32; o <<= 1) {
+    float a2[8];
+    const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
+    const float l2 = __shfl_xor_sync(0xffffffffu, l, o);
+#pragma unroll
+    for (int c = 0; c < 8; ++c) a2[c] = __shfl_xor_sync(0xffffffffu, a[c], o);
+    fold(m, l, a, m2, l2, a2);
   }
-  float m = -INFINITY, l = 0.f, acc[8];
-#pragma unroll
-  for (int c = 0; c < 8; ++c) acc[c] = 0.f;
+}
 
-  if (stream_query(q_sid, L.P_max)) {
-    const int seg = q_sid - 1;
-    int n = L.len[seg];
-    n = n < L.S_cap ? n : L.S_cap;
-    const uint4* kb = reinterpret_cast<const uint4*>(L.k_suf) + ((int64_t)seg * L.H + h) * L.S_cap * LPK;
-    const uint4* vb = reinterpret_cast<const uint4*>(L.v_suf) + ((int64_t)seg * L.H + h) * L.S_cap * LPK;
-    const int16_t* sb = L.sid + (int64_t)seg * L.S_cap;
-    const int32_t* pb = L.pos + (int64_t)seg * L.S_cap;
-    for (int t0 = 0; t0 < n; t0 += KPI * U) {
-      uint4 kk[U], vv[U];
-      bool vis[U];
+// Warp-uniform bounded wait on a stage barrier.
+__device__ __forceinline__ bool stage_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                           long long limit, int32_t* status, int lane) {
+  const long long t0 = clock64();
+  while (true) {
+    const bool done = mbar_try_wait(bar, parity);
+    if (__all_sync(0xffffffffu, done)) return true;
+    int stop = 0;
+    if (lane == 0) {
+      if (*abort_flag) {
+        stop = 1;
+      } else if (clock64() - t0 > limit) {
+        *abort_flag = 1;
+        set_status(status, PP_DEV_TIMEOUT);
+        stop = 1;
+      }
+    }
+    if (__shfl_sync(0xffffffffu, stop, 0)) return false;
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(SufCfg<D>::WARPS * 32) suffix_merge(const SufParams p) {
+  using C = SufCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) &
+                                             ~uintptr_t(127));
+  __shared__ uint64_t bars[C::WARPS][C::NS];
+  __shared__ int abort_sh;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane / C::LPK, j = lane % C::LPK;
+  uint8_t* ring = smem + warp * C::NS * C::STAGE;
+  ItemRec* tbl = reinterpret_cast<ItemRec*>(smem + C::WARPS * C::NS * C::STAGE) + warp * C::TBL;
+  uint64_t* full = bars[warp];
+  if (threadIdx.x == 0) abort_sh = 0;
+  if (lane == 0) {
+    for (int i = 0; i < C::NS; ++i) mbar_init(full + i, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  volatile int* abort_flag = &abort_sh;
+
+  // This warp's items: a contiguous, balanced block of the (head, row) space
+  // (head-major, so in a prefill neighbouring items share a segment).
+  const int64_t items = (int64_t)p.rows * p.H;
+  const int64_t gw = (int64_t)blockIdx.x * C::WARPS + warp;
+  const int64_t GW = (int64_t)gridDim.x * C::WARPS;
+  const int64_t i_begin = gw * items / GW, i_end = (gw + 1) * items / GW;
+  const size_t seg_elems = (size_t)p.S_cap * D;
+
+  uint32_t issued = 0, consumed = 0;
+  bool ok = true;
+  for (int64_t r0 = i_begin; ok && r0 < i_end; r0 += C::TBL) {
+    const int cnt = (int)min((int64_t)C::TBL, i_end - r0);
+    // ---- item table of this round: two parallel gathers instead of one
+    // dependent chain per item
+    for (int k = lane; k < cnt; k += 32) {
+      const int64_t item = r0 + k;
+      const int r = (int)(item % p.rows);
+      const int s = p.q_sid[r];
+      ItemRec rec;
+      rec.qp = p.q_pos[r];
+      rec.s = stream_query(s, p.P_max) ? s : 0;
+      rec.n = 0;
+      rec.pad = s;
+      tbl[k] = rec;
+    }
+    __syncwarp();
+    for (int k = lane; k < cnt; k += 32) {
+      const int s = tbl[k].s;
+      if (s) {
+        const int n = p.len[s - 1];
+        tbl[k].n = n < p.S_cap ? n : p.S_cap;
+      }
+    }
+    __syncwarp();
+
+    // Producer cursor over (item, first key) chunks of this round.
+    int pk = 0, pt0 = 0;
+    auto issue_next = [&](uint32_t stage) -> bool {
+      while (pk < cnt && pt0 >= tbl[pk].n) {
+        ++pk;
+        pt0 = 0;
+      }
+      if (pk >= cnt) return false;
+      if (lane == 0) {
+        const ItemRec rec = tbl[pk];
+        const int h = (int)((r0 + pk) / p.rows);
+        const int nk = min(C::CK, rec.n - pt0);
+        const size_t off = ((size_t)(rec.s - 1) * p.H + h) * seg_elems + (size_t)pt0 * D;
+        uint8_t* st = ring + stage * C::STAGE;
+        fence_proxy_async();
+        mbar_arrive_expect_tx(full + stage, 2u * nk * C::ROW);
+        bulk_load(st, p.k_suf + off, nk * C::ROW, full + stage);
+        bulk_load(st + C::HALF, p.v_suf + off, nk * C::ROW, full + stage);
+      }
+      pt0 += C::CK;
+      return true;
+    };
+    for (int i = 0; i < C::NS - 1; ++i)
+      if (issue_next(issued % C::NS)) ++issued;
+
+    for (int k = 0; k < cnt; ++k) {
+      const int64_t item = r0 + k;
+      const int h = (int)(item / p.rows), r = (int)(item - (int64_t)h * p.rows);
+      const ItemRec rec = tbl[k];
+      const bool valid = rec.s != 0;
+      // query fragment, and the document partials of this (row, head), fetched now
+      // so their latency hides behind the segment's chunks
+      const uint4 qv = reinterpret_cast<const uint4*>(p.q + ((int64_t)r * p.H + h) * D)[j];
+      int c0 = 0, c1 = -1;
+      int64_t slot0 = 0;
+      const int rr = r % kGroupRows;
+      if (valid && p.has_doc) {
+        const int u = (r / kGroupRows) * p.H + h;
+        c0 = plan_cta_of(p.plan, (int64_t)u * p.plan.T);
+        c1 = plan_cta_of(p.plan, (int64_t)u * p.plan.T + p.plan.T - 1);
+        slot0 = (int64_t)u * p.plan.max_chunks;
+      }
+      float2 pre_ml[C::PRE];
+      float4 pre_o[C::PRE][2];
 #pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int t = t0 + u * KPI + g;
-        vis[u] = false;
-        if (t < n) {
-          kk[u] = __ldg(kb + (int64_t)t * LPK + j);
-          vv[u] = __ldg(vb + (int64_t)t * LPK + j);
-          vis[u] = slot_visible(q_sid, q_pos, __ldg(sb + t), __ldg(pb + t), t, n);
+      for (int e = 0; e < C::PRE; ++e) {
+        const int c = c0 + g + e * C::KPI;
+        if (c <= c1) {
+          const int64_t sl = (slot0 + c - c0) * kGroupRows + rr;
+          pre_ml[e] = *reinterpret_cast<const float2*>(p.doc_ml + sl * 2);
+          const float4* src = reinterpret_cast<const float4*>(p.doc_o + sl * D + j * 8);
+          pre_o[e][0] = src[0];
+          pre_o[e][1] = src[1];
         }
       }
-      float x[U];
+      float qf[8];
+      {
+        const uint32_t w[4] = {qv.x, qv.y, qv.z, qv.w};
 #pragma unroll
-      for (int u = 0; u < U; ++u) {
-        float dot = 0.f;
-        if (t0 + u * KPI < n) {  // warp-uniform: some group has a key here
-          const uint32_t w[4] = {kk[u].x, kk[u].y, kk[u].z, kk[u].w};
+        for (int c = 0; c < 4; ++c) {
+          const float2 f = bf2_to_f2(w[c]);
+          qf[2 * c] = f.x * p.sl2;
+          qf[2 * c + 1] = f.y * p.sl2;
+        }
+      }
+      float m = -INFINITY, l = 0.f, acc[8];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) acc[c] = 0.f;
+      const int16_t* sb = p.sid + (size_t)(valid ? rec.s - 1 : 0) * p.S_cap;
+      const int32_t* pb = p.pos + (size_t)(valid ? rec.s - 1 : 0) * p.S_cap;
+
+      for (int t0 = 0; t0 < rec.n; t0 += C::CK) {
+        if (issue_next(issued % C::NS)) ++issued;
+        const int nk = min(C::CK, rec.n - t0);
+        int tsid = -1, tpos = 0;  // this chunk's tags, one per lane (loaded before the wait)
+        if (lane < nk) {
+          tsid = __ldg(sb + t0 + lane);
+          tpos = __ldg(pb + t0 + lane);
+        }
+        const uint32_t stage = consumed % C::NS;
+        if (!(ok = stage_wait(full + stage, (consumed / C::NS) & 1, abort_flag, p.wait_limit,
+                              p.status, lane)))
+          break;
+        const uint8_t* sK = ring + stage * C::STAGE;
+        const uint8_t* sV = sK + C::HALF;
+        float x[C::CK / C::KPI];
+#pragma unroll
+        for (int u = 0; u < C::CK / C::KPI; ++u) {
+          const int kk = u * C::KPI + g;
+          const uint4 kv = *reinterpret_cast<const uint4*>(sK + kk * C::ROW + j * 16);
+          const uint32_t w[4] = {kv.x, kv.y, kv.z, kv.w};
+          float dot = 0.f;
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
             const float2 f = bf2_to_f2(w[c]);
@@ -75,101 +274,150 @@ __device__ __forceinline__ void segment_partial(const pp_kv_layer& L, const uint
             dot = fmaf(qf[2 * c + 1], f.y, dot);
           }
 #pragma unroll
-          for (int o = 1; o < LPK; o <<= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+          for (int o = 1; o < C::LPK; o <<= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+          const int ks = __shfl_sync(0xffffffffu, tsid, kk);
+          const int kp = __shfl_sync(0xffffffffu, tpos, kk);
+          x[u] = (kk < nk && slot_visible(rec.s, rec.qp, ks, kp, t0 + kk, rec.n)) ? dot : -INFINITY;
         }
-        x[u] = vis[u] ? dot : -INFINITY;
+        float cm = m;
+#pragma unroll
+        for (int u = 0; u < C::CK / C::KPI; ++u) cm = fmaxf(cm, x[u]);
+        if (cm != -INFINITY) {
+          const float corr = exp2f(m - cm);
+          l *= corr;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) acc[c] *= corr;
+#pragma unroll
+          for (int u = 0; u < C::CK / C::KPI; ++u) {
+            // masked keys are skipped, not weighted by 0: stage rows past the
+            // chunk's end hold stale shared memory
+            if (x[u] == -INFINITY) continue;
+            const float pr = exp2f(x[u] - cm);
+            l += pr;
+            const int kk = u * C::KPI + g;
+            const uint4 vv = *reinterpret_cast<const uint4*>(sV + kk * C::ROW + j * 16);
+            const uint32_t w[4] = {vv.x, vv.y, vv.z, vv.w};
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              const float2 f = bf2_to_f2(w[c]);
+              acc[2 * c] = fmaf(pr, f.x, acc[2 * c]);
+              acc[2 * c + 1] = fmaf(pr, f.y, acc[2 * c + 1]);
+            }
+          }
+          m = cm;
+        }
+        __syncwarp();
+        ++consumed;
       }
-      float cm = m;
+      if (!ok) break;
+
+      // ---- merge with the document partials of (row, head)
+      combine_groups<C::LPK>(m, l, acc);
+      if (g != 0) {  // group 0 carries the suffix partial, the others start empty
+        m = -INFINITY;
+        l = 0.f;
 #pragma unroll
-      for (int u = 0; u < U; ++u) cm = fmaxf(cm, x[u]);
-      if (cm == -INFINITY) continue;  // nothing visible yet for this lane group
-      const float corr = exp2f(m - cm);  // m = -inf gives 0
-      l *= corr;
+        for (int c = 0; c < 8; ++c) acc[c] = 0.f;
+      }
 #pragma unroll
-      for (int c = 0; c < 8; ++c) acc[c] *= corr;
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        if (!vis[u]) continue;
-        const float p = exp2f(x[u] - cm);
-        l += p;
-        const uint32_t w[4] = {vv[u].x, vv[u].y, vv[u].z, vv[u].w};
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const float2 f = bf2_to_f2(w[c]);
-          acc[2 * c] = fmaf(p, f.x, acc[2 * c]);
-          acc[2 * c + 1] = fmaf(p, f.y, acc[2 * c + 1]);
+      for (int e = 0; e < C::PRE; ++e) {
+        if (c0 + g + e * C::KPI <= c1) {
+          const float a2[8] = {pre_o[e][0].x, pre_o[e][0].y, pre_o[e][0].z, pre_o[e][0].w,
+                               pre_o[e][1].x, pre_o[e][1].y, pre_o[e][1].z, pre_o[e][1].w};
+          fold(m, l, acc, pre_ml[e].x, pre_ml[e].y, a2);
         }
       }
-      m = cm;
+      for (int c = c0 + g + C::PRE * C::KPI; c <= c1; c += C::KPI) {
+        const int64_t sl = (slot0 + c - c0) * kGroupRows + rr;
+        const float2 ml = *reinterpret_cast<const float2*>(p.doc_ml + sl * 2);
+        const float4* src = reinterpret_cast<const float4*>(p.doc_o + sl * D + j * 8);
+        const float4 a0 = src[0], a1 = src[1];
+        const float a2[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+        fold(m, l, acc, ml.x, ml.y, a2);
+      }
+      combine_groups<C::LPK>(m, l, acc);
+      const bool any = valid && l > 0.f;
+      const float inv = any ? 1.f / l : 0.f;
+      if (g == 0) {
+        uint4 pkd;
+        pkd.x = f2_to_bf2(acc[0] * inv, acc[1] * inv);
+        pkd.y = f2_to_bf2(acc[2] * inv, acc[3] * inv);
+        pkd.z = f2_to_bf2(acc[4] * inv, acc[5] * inv);
+        pkd.w = f2_to_bf2(acc[6] * inv, acc[7] * inv);
+        reinterpret_cast<uint4*>(p.o + ((int64_t)r * p.H + h) * D)[j] = pkd;
+      }
+      if (lane == 0) {
+        if (p.lse) p.lse[(int64_t)r * p.H + h] = any ? (m + log2f(l)) * kLn2 : -INFINITY;
+        if (h == 0 && (rec.pad == 0 || rec.pad > p.P_max)) set_status(p.status, PP_DEV_BAD_STREAM);
+      }
     }
+    __syncwarp();
   }
-  // Combine the KPI key groups of the warp.
-#pragma unroll
-  for (int o = LPK; o < 32; o <<= 1) {
-    const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
-    const float l2 = __shfl_xor_sync(0xffffffffu, l, o);
-    const float mm = fmaxf(m, m2);
-    const float a = (m == -INFINITY) ? 0.f : exp2f(m - mm);
-    const float b = (m2 == -INFINITY) ? 0.f : exp2f(m2 - mm);
-    l = l * a + l2 * b;
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      const float a2 = __shfl_xor_sync(0xffffffffu, acc[c], o);
-      acc[c] = acc[c] * a + a2 * b;
-    }
-    m = mm;
-  }
-  if (g == 0) {
-    float4* dst = reinterpret_cast<float4*>(out_o + ((int64_t)r * L.H + h) * D + j * 8);
-    dst[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
-    dst[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
-  }
-  if (lane == 0) {
-    out_ml[((int64_t)r * L.H + h) * 2 + 0] = m;
-    out_ml[((int64_t)r * L.H + h) * 2 + 1] = l;
+  // Drain: copies issued ahead that no item consumed (only after an abort).
+  if (!ok && lane == 0) {
+    volatile int never = 0;
+    for (uint32_t c = consumed; c < issued; ++c)
+      mbar_wait(full + c % C::NS, (c / C::NS) & 1, &never, p.wait_limit, nullptr);
   }
 }
 
-// Warp w handles head w / rows and row w % rows (head-major, so the warps of
-// one CTA share a head and, in a prefill, mostly a stream segment).
-template <int D>
-__global__ void __launch_bounds__(256) suffix_pass(pp_kv_layer L, const uint16_t* __restrict__ q,
-                                                   const int16_t* __restrict__ q_sid,
-                                                   const int32_t* __restrict__ q_pos, int rows,
-                                                   float sl2, float* __restrict__ out_o,
-                                                   float* __restrict__ out_ml) {
-  const int64_t w = (int64_t)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
-  if (w >= (int64_t)rows * L.H) return;
-  const int h = (int)(w / rows), r = (int)(w - (int64_t)h * rows);
-  const int lane = threadIdx.x & 31;
-  const int s = q_sid[r];
-  if (lane == 0 && h == 0 && (s == 0 || s > L.P_max)) set_status(L.status, PP_DEV_BAD_STREAM);
-  segment_partial<D>(L, q, r, h, s, q_pos[r], sl2, out_o, out_ml, lane);
-}
-
-cudaError_t launch_suffix_pass(const pp_kv_layer& L, const uint16_t* q, const int16_t* q_sid,
-                               const int32_t* q_pos, int rows, float scale, const Partials& part,
-                               cudaStream_t st) {
-  const int64_t warps = (int64_t)rows * L.H;
-  const int blocks = (int)((warps + 7) / 8);
-  const float sl2 = scale * kLog2e;
-  if (L.d == 128)
-    suffix_pass<128><<<blocks, 256, 0, st>>>(L, q, q_sid, q_pos, rows, sl2, part.suf_o, part.suf_ml);
-  else
-    suffix_pass<64><<<blocks, 256, 0, st>>>(L, q, q_sid, q_pos, rows, sl2, part.suf_o, part.suf_ml);
-  return cudaGetLastError();
+cudaError_t launch_suffix_merge(const pp_kv_layer& L, const uint16_t* q, const int16_t* q_sid,
+                                const int32_t* q_pos, int rows, float scale, const SplitPlan& plan,
+                                bool has_doc, const Partials& part, uint16_t* o, float* lse,
+                                long long wait_limit, int num_sms, cudaStream_t st) {
+  SufParams prm;
+  prm.rows = rows;
+  prm.H = L.H;
+  prm.P_max = L.P_max;
+  prm.S_cap = L.S_cap;
+  prm.q = q;
+  prm.q_sid = q_sid;
+  prm.q_pos = q_pos;
+  prm.k_suf = L.k_suf;
+  prm.v_suf = L.v_suf;
+  prm.sid = L.sid;
+  prm.pos = L.pos;
+  prm.len = L.len;
+  prm.status = L.status;
+  prm.sl2 = scale * kLog2e;
+  prm.plan = plan;
+  prm.has_doc = has_doc ? 1 : 0;
+  prm.doc_o = part.doc_o;
+  prm.doc_ml = part.doc_ml;
+  prm.o = o;
+  prm.lse = lse;
+  prm.wait_limit = wait_limit;
+  const int64_t items = (int64_t)rows * L.H;
+  auto go = [&](auto kernel, int warps, int smem, std::atomic<uint64_t>& ready) -> cudaError_t {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const uint64_t bit = 1ull << (dev & 63);
+    if (!(ready.load() & bit)) {  // once per device
+      e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      if (e != cudaSuccess) return e;
+      ready.fetch_or(bit);
+    }
+    int64_t ctas = (items + warps - 1) / warps;
+    if (ctas > num_sms) ctas = num_sms;
+    kernel<<<(int)ctas, warps * 32, smem, st>>>(prm);
+    return cudaGetLastError();
+  };
+  static std::atomic<uint64_t> ready128{0}, ready64{0};
+  if (L.d == 128) return go(suffix_merge<128>, SufCfg<128>::WARPS, SufCfg<128>::SMEM, ready128);
+  return go(suffix_merge<64>, SufCfg<64>::WARPS, SufCfg<64>::SMEM, ready64);
 }
 
 // K6 (ablation): the document read once PER QUERY ROW -- one warp per (row,
 // head) over all doc_len keys, no tensor cores.  This is what serving each
 // question as its own request costs (the page's "Inside decode step":
 // batched requests read the document keys once per question).  Writes the
-// document partial of chunk 0 of unit (row / kGroupRows) * H + h, so the
-// same merge kernel finishes it; the plan it pairs with has one chunk per unit.
+// document partial of chunk 0 of unit (row / kGroupRows) * H + h, which the
+// suffix kernel's merge then finishes; the plan it pairs with has one chunk
+// per unit.
 template <int D>
 __global__ void __launch_bounds__(256) doc_per_stream(pp_kv_layer L, int doc_len,
-                                                      const uint16_t* __restrict__ q,
-                                                      const int16_t* __restrict__ q_sid, int rows,
+                                                      const uint16_t* __restrict__ q, int rows,
                                                       float sl2, int max_chunks,
                                                       float* __restrict__ doc_o,
                                                       float* __restrict__ doc_ml) {
@@ -232,34 +480,19 @@ __global__ void __launch_bounds__(256) doc_per_stream(pp_kv_layer L, int doc_len
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       if (x[u] == -INFINITY) continue;
-      const float p = exp2f(x[u] - cm);
-      l += p;
+      const float pr = exp2f(x[u] - cm);
+      l += pr;
       const uint32_t wv[4] = {vv[u].x, vv[u].y, vv[u].z, vv[u].w};
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         const float2 f = bf2_to_f2(wv[c]);
-        acc[2 * c] = fmaf(p, f.x, acc[2 * c]);
-        acc[2 * c + 1] = fmaf(p, f.y, acc[2 * c + 1]);
+        acc[2 * c] = fmaf(pr, f.x, acc[2 * c]);
+        acc[2 * c + 1] = fmaf(pr, f.y, acc[2 * c + 1]);
       }
     }
     m = cm;
   }
-#pragma unroll
-  for (int o = LPK; o < 32; o <<= 1) {
-    const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
-    const float l2 = __shfl_xor_sync(0xffffffffu, l, o);
-    const float mm = fmaxf(m, m2);
-    const float a = (m == -INFINITY) ? 0.f : exp2f(m - mm);
-    const float b = (m2 == -INFINITY) ? 0.f : exp2f(m2 - mm);
-    l = l * a + l2 * b;
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      const float a2 = __shfl_xor_sync(0xffffffffu, acc[c], o);
-      acc[c] = acc[c] * a + a2 * b;
-    }
-    m = mm;
-  }
-  (void)q_sid;
+  combine_groups<LPK>(m, l, acc);
   const int64_t slot = ((int64_t)(r / kGroupRows) * L.H + h) * max_chunks;
   const int rr = r % kGroupRows;
   if (g == 0) {
@@ -267,24 +500,21 @@ __global__ void __launch_bounds__(256) doc_per_stream(pp_kv_layer L, int doc_len
     dst[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
     dst[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
   }
-  if (lane == 0) {
-    doc_ml[(slot * kGroupRows + rr) * 2 + 0] = m;
-    doc_ml[(slot * kGroupRows + rr) * 2 + 1] = l;
-  }
+  if (lane == 0) reinterpret_cast<float2*>(doc_ml)[slot * kGroupRows + rr] = make_float2(m, l);
 }
 
-cudaError_t launch_doc_per_stream(const pp_kv_layer& L, int doc_len, const uint16_t* q,
-                                  const int16_t* q_sid, int rows, float scale, int max_chunks,
-                                  const Partials& part, cudaStream_t st) {
+cudaError_t launch_doc_per_stream(const pp_kv_layer& L, int doc_len, const uint16_t* q, int rows,
+                                  float scale, int max_chunks, const Partials& part,
+                                  cudaStream_t st) {
   const int64_t warps = (int64_t)rows * L.H;
   const int blocks = (int)((warps + 7) / 8);
   const float sl2 = scale * kLog2e;
   if (L.d == 128)
-    doc_per_stream<128><<<blocks, 256, 0, st>>>(L, doc_len, q, q_sid, rows, sl2, max_chunks,
-                                                part.doc_o, part.doc_ml);
+    doc_per_stream<128><<<blocks, 256, 0, st>>>(L, doc_len, q, rows, sl2, max_chunks, part.doc_o,
+                                                part.doc_ml);
   else
-    doc_per_stream<64><<<blocks, 256, 0, st>>>(L, doc_len, q, q_sid, rows, sl2, max_chunks,
-                                               part.doc_o, part.doc_ml);
+    doc_per_stream<64><<<blocks, 256, 0, st>>>(L, doc_len, q, rows, sl2, max_chunks, part.doc_o,
+                                               part.doc_ml);
   return cudaGetLastError();
 }
 

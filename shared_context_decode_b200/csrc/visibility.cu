@@ -1,4 +1,4 @@
-// Test aid: evaluates, on the device, the same slot predicate the suffix
+// Test aids.  visibility_kernel evaluates, on the device, the same slot predicate the suffix
 // pass applies (common.cuh, slot_visible), over every segment slot of the
 // cache, so tests can compare "which keys each query sees" bit for bit.
 #include "common.cuh"
@@ -43,6 +43,27 @@ cudaError_t launch_visibility(const pp_kv_layer& L, int doc_len, const int16_t* 
                               const int32_t* q_pos, int nq, int32_t* count_out, uint8_t* mask_out,
                               cudaStream_t st) {
   visibility_kernel<<<nq, 256, 0, st>>>(L, doc_len, q_sid, q_pos, count_out, mask_out);
+  return cudaGetLastError();
+}
+
+// Test aid: both exponentials the document pass uses, element-wise.
+__global__ void exp2_kernel(const float* __restrict__ x, float* __restrict__ y_poly,
+                            float* __restrict__ y_hw, int n) {
+  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (i >= n) return;
+  const float2 v = make_float2(x[i], i + 1 < n ? x[i + 1] : 0.f);
+  const float2 r = ex2_poly2(v);
+  y_poly[i] = r.x;
+  y_hw[i] = ex2_mufu(v.x);
+  if (i + 1 < n) {
+    y_poly[i + 1] = r.y;
+    y_hw[i + 1] = ex2_mufu(v.y);
+  }
+}
+
+cudaError_t launch_exp2(const float* x, float* y_poly, float* y_hw, int n, cudaStream_t st) {
+  const int pairs = (n + 1) / 2;
+  exp2_kernel<<<(pairs + 255) / 256, 256, 0, st>>>(x, y_poly, y_hw, n);
   return cudaGetLastError();
 }
 

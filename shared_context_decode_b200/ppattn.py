@@ -43,7 +43,24 @@ class LayerStruct(ctypes.Structure):
 
 class Options(ctypes.Structure):
     _fields_ = [("splits", _i32), ("ablation_doc_per_stream", _i32),
-                ("debug_inject_timeout", _i32), ("wait_limit_log2", _i32)]
+                ("debug_inject_timeout", _i32), ("wait_limit_log2", _i32),
+                ("events", ctypes.POINTER(_vp))]
+
+    def set_events(self, events):
+        """Record 3 CUDA events (torch.cuda.Event, enable_timing=True) around
+        the kernels of each decode/prefill call -- before the document pass,
+        after it, after the suffix pass with its merge; None clears them."""
+        if events is None:
+            self.events = None
+            self._ev = None
+            return
+        for e in events:
+            if e.cuda_event == 0:   # torch creates the event on first record
+                e.record()
+        if len(events) != 3:
+            raise ValueError("set_events takes 3 events")
+        self._ev = (_vp * 3)(*[e.cuda_event for e in events])
+        self.events = ctypes.cast(self._ev, ctypes.POINTER(_vp))
 
 
 _LP = ctypes.POINTER(LayerStruct)
@@ -68,6 +85,7 @@ _decode = _sig("pp_decode_attn", _i32, _LP, _i32, _vp, _vp, _vp, _i32, ctypes.c_
 _prefill = _sig("pp_prefill_attn", _i32, _LP, _i32, _vp, _vp, _vp, _i32, ctypes.c_float, _vp,
                 _vp, _vp, _sz, _OP, _vp)
 _visibility = _sig("pp_debug_visibility", _i32, _LP, _i32, _vp, _vp, _i32, _vp, _vp, _vp)
+_exp2 = _sig("pp_debug_exp2", _i32, _vp, _vp, _vp, _i32, _vp)
 _dev_status = _sig("pp_get_device_status", _i32, _LP, ctypes.POINTER(_i32), _vp)
 _split_plan = _sig("pp_debug_split_plan", _i32, _i32, _i32, _i32, _i32,
                    ctypes.POINTER(ctypes.c_int64), _i32)
@@ -75,7 +93,7 @@ _split_plan = _sig("pp_debug_split_plan", _i32, _i32, _i32, _i32, _i32,
 EXPORTED = ("pp_status_str", "pp_abi_version", "pp_kv_reset", "pp_kv_append",
             "pp_decode_workspace_bytes", "pp_prefill_workspace_bytes", "pp_decode_attn",
             "pp_prefill_attn", "pp_debug_visibility", "pp_get_device_status",
-            "pp_debug_split_plan")
+            "pp_debug_split_plan", "pp_debug_exp2")
 
 
 class PPError(RuntimeError):
@@ -129,7 +147,8 @@ class KVLayer:
     status [1] int32.
     """
 
-    def __init__(self, H: int, d: int, doc_cap: int, P_max: int, S_cap: int, device="cuda"):
+    def __init__(self, H: int, d: int, doc_cap: int, P_max: int, S_cap: int, device="cuda",
+                 len_buf: Optional[torch.Tensor] = None):
         dev = torch.device(device)
         if dev.type == "cuda" and dev.index is None:
             dev = torch.device("cuda", torch.cuda.current_device())
@@ -142,7 +161,14 @@ class KVLayer:
         self.v_suf = torch.zeros((P_max, H, S_cap, d), dtype=bf, device=dev)
         self.sid = torch.zeros((P_max, S_cap), dtype=torch.int16, device=dev)
         self.pos = torch.zeros((P_max, S_cap), dtype=torch.int32, device=dev)
-        self.len = torch.zeros((P_max,), dtype=torch.int32, device=dev)
+        if len_buf is not None:      # caller-provided view, e.g. one row of [layers, P_max]
+            _want(len_buf, torch.int32, "len_buf", dev)
+            if len_buf.shape != (P_max,):
+                raise ValueError("len_buf must be [P_max] int32")
+            len_buf.zero_()
+            self.len = len_buf
+        else:
+            self.len = torch.zeros((P_max,), dtype=torch.int32, device=dev)
         self.status = torch.zeros((1,), dtype=torch.int32, device=dev)
         self.struct = LayerStruct(H, d, doc_cap, P_max, S_cap, 0,
                                   self.k_doc.data_ptr(), self.v_doc.data_ptr(),
@@ -247,6 +273,15 @@ def debug_visibility(layer: KVLayer, doc_len: int, q_sid: torch.Tensor, q_pos: t
     _check(_visibility(layer.ref, doc_len, _ptr(q_sid), _ptr(q_pos), nq, _ptr(count), _ptr(mask),
                        _stream(dev)), "pp_debug_visibility")
     return count, mask
+
+
+def debug_exp2(x: torch.Tensor):
+    """(polynomial 2^x, hardware 2^x) for a float32 CUDA tensor x."""
+    if x.dtype != torch.float32 or not x.is_cuda or not x.is_contiguous():
+        raise TypeError("x must be a contiguous float32 CUDA tensor")
+    yp, yh = torch.empty_like(x), torch.empty_like(x)
+    _check(_exp2(_ptr(x), _ptr(yp), _ptr(yh), x.numel(), _stream(x.device)), "pp_debug_exp2")
+    return yp, yh
 
 
 def device_status(layer: KVLayer) -> int:

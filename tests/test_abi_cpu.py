@@ -97,11 +97,11 @@ def test_workspace_sizes_with_explicit_split(pp):
     ws = pp.decode_workspace_bytes(256, 32, 128, 16384, opt)
     plan = pp.split_plan(256, 32, 16384, 148)
     slots = plan["units"] * plan["max_chunks"] * 256
-    expect = slots * 128 * 4 + slots * 2 * 4 + 256 * 32 * 128 * 4 + 256 * 32 * 2 * 4
+    expect = slots * 128 * 4 + slots * 2 * 4       # document partials (O; max and sum)
     assert ws == expect
     assert pp.decode_workspace_bytes(4, 4, 96, 10, opt) == 0
-    # no document: only the suffix partials
-    assert pp.decode_workspace_bytes(8, 2, 64, 0, opt) == 8 * 2 * 64 * 4 + 256
+    # no document: nothing to carry between kernels
+    assert pp.decode_workspace_bytes(8, 2, 64, 0, opt) == 0
 
 
 @pytest.mark.parametrize("rows,H,doc_len,ctas", [
