@@ -174,6 +174,34 @@ pp_status pp_decode_attn(const pp_kv_layer *layer, int32_t doc_len, const uint16
                          uint16_t *o, float *lse, void *ws, size_t ws_bytes,
                          const pp_options *opt, void *stream);
 
+/*
+ * pp_decode_attn for callers that cannot allocate device memory.  The pages
+ * have no counterpart: this is a library convenience.
+ *
+ * Some callers cannot obtain a workspace -- for example a plugin inside a host
+ * application that owns all device memory and gives the plugin no allocator,
+ * or a serving loop that forbids device allocation after start-up because
+ * cudaMalloc can synchronise the device.  This call takes the same arguments
+ * as pp_decode_attn minus the workspace; the caller still passes q, the tags,
+ * o and lse.  The document pass's partials go to a scratch array built into
+ * the library (PP_NOALLOC_SCRATCH_BYTES on every GPU that loads it, held until
+ * the process exits).  It allocates nothing.
+ *   - Returns PP_ERR_CAPACITY, launching nothing, when the call would need
+ *     more than PP_NOALLOC_SCRATCH_BYTES (pp_decode_workspace_bytes tells how
+ *     much it needs; 32 MiB covers P = 256, H = 32, d = 128, doc 16384 on a
+ *     148-SM B200).
+ *   - The first call on each device looks up the scratch address on that
+ *     device (make it the current device); make that first call before any
+ *     stream capture.
+ *   - Every call shares the one scratch array: calls whose kernels overlap on
+ *     the GPU (different streams, unordered) corrupt each other's results.
+ */
+#define PP_NOALLOC_SCRATCH_BYTES (32u << 20)
+pp_status pp_decode_attn_noalloc(const pp_kv_layer *layer, int32_t doc_len, const uint16_t *q,
+                                 const int16_t *q_sid, const int32_t *q_pos, int32_t P,
+                                 float scale, uint16_t *o, float *lse, const pp_options *opt,
+                                 void *stream);
+
 /* Workspace bytes pp_prefill_attn needs for R question rows. */
 size_t pp_prefill_workspace_bytes(int32_t R, int32_t H, int32_t d, int32_t doc_len,
                                   const pp_options *opt);

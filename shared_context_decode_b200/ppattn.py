@@ -82,6 +82,8 @@ _dec_ws = _sig("pp_decode_workspace_bytes", _sz, _i32, _i32, _i32, _i32, _OP)
 _pre_ws = _sig("pp_prefill_workspace_bytes", _sz, _i32, _i32, _i32, _i32, _OP)
 _decode = _sig("pp_decode_attn", _i32, _LP, _i32, _vp, _vp, _vp, _i32, ctypes.c_float, _vp, _vp,
                _vp, _sz, _OP, _vp)
+_decode_noalloc = _sig("pp_decode_attn_noalloc", _i32, _LP, _i32, _vp, _vp, _vp, _i32,
+                      ctypes.c_float, _vp, _vp, _OP, _vp)
 _prefill = _sig("pp_prefill_attn", _i32, _LP, _i32, _vp, _vp, _vp, _i32, ctypes.c_float, _vp,
                 _vp, _vp, _sz, _OP, _vp)
 _visibility = _sig("pp_debug_visibility", _i32, _LP, _i32, _vp, _vp, _i32, _vp, _vp, _vp)
@@ -93,7 +95,10 @@ _split_plan = _sig("pp_debug_split_plan", _i32, _i32, _i32, _i32, _i32,
 EXPORTED = ("pp_status_str", "pp_abi_version", "pp_kv_reset", "pp_kv_append",
             "pp_decode_workspace_bytes", "pp_prefill_workspace_bytes", "pp_decode_attn",
             "pp_prefill_attn", "pp_debug_visibility", "pp_get_device_status",
-            "pp_debug_split_plan", "pp_debug_exp2")
+            "pp_debug_split_plan", "pp_debug_exp2", "pp_decode_attn_noalloc")
+
+# Size of the scratch array built into the library for pp_decode_attn_noalloc.
+NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
 class PPError(RuntimeError):
@@ -248,6 +253,32 @@ def decode_attn(layer: KVLayer, doc_len: int, q: torch.Tensor, q_sid: torch.Tens
     """Decode-step attention of P query rows; returns o [P, H, d] bf16."""
     return _attn(_decode, "pp_decode_attn", layer, doc_len, q, q_sid, q_pos, scale, o, lse, ws,
                  opt, decode_workspace_bytes)
+
+
+def decode_attn_noalloc(layer: KVLayer, doc_len: int, q: torch.Tensor, q_sid: torch.Tensor,
+                        q_pos: torch.Tensor, scale: float, o: Optional[torch.Tensor] = None,
+                        lse: Optional[torch.Tensor] = None,
+                        opt: Optional[Options] = None) -> torch.Tensor:
+    """decode_attn without a workspace, for callers that cannot allocate
+    device memory (the library's built-in scratch holds the partials).  Pass
+    `o` to avoid the one torch allocation this wrapper would otherwise make.
+    Calls must not overlap on the GPU: they share the scratch."""
+    dev = layer.device
+    rows = q_sid.shape[0]
+    _want(q, torch.bfloat16, "q", dev)
+    _want(q_sid, torch.int16, "q_sid", dev)
+    _want(q_pos, torch.int32, "q_pos", dev)
+    if q.shape != (rows, layer.H, layer.d) or q_pos.shape != (rows,):
+        raise ValueError("pp_decode_attn_noalloc: q must be [rows, H, d], q_sid and q_pos [rows]")
+    if o is None:
+        o = torch.empty_like(q)
+    _want(o, torch.bfloat16, "o", dev)
+    if lse is not None:
+        _want(lse, torch.float32, "lse", dev)
+    _check(_decode_noalloc(layer.ref, doc_len, _ptr(q), _ptr(q_sid), _ptr(q_pos), rows,
+                           float(scale), _ptr(o), _ptr(lse), _opts(opt), _stream(dev)),
+           "pp_decode_attn_noalloc")
+    return o
 
 
 def prefill_attn(layer: KVLayer, doc_len: int, q: torch.Tensor, q_sid: torch.Tensor,
