@@ -172,16 +172,16 @@ class DecodeStep:
         self.ws = pp.workspace(pp.decode_workspace_bytes(W.P, W.H, W.d, W.N), device)
         self.graph = None
 
-    def run_eager(self, opt=None, layer_events=None):
+    def run_eager(self, opts=None):
+        """One decode step, launched eagerly (also the body that is captured);
+        opts: per-layer pp_options or None."""
         pp = self.pp
         self.len_all.copy_(self.len0)
         for l in range(self.layers):
             x = self.inp[l]
             pp.kv_append(self.cache[l], x["k"], x["v"], x["sid"], x["pos"])
-            if layer_events is not None:
-                opt.set_events(layer_events[l])
             pp.decode_attn(self.cache[l], self.W.N, x["q"], x["sid"], x["pos"], self.W.scale,
-                           o=x["o"], ws=self.ws, opt=opt)
+                           o=x["o"], ws=self.ws, opt=None if opts is None else opts[l])
 
     def capture(self):
         self.run_eager()           # warm: per-device setup happens outside the capture
@@ -230,20 +230,35 @@ def load_peaks():
 
 
 def measure_doc_pass(step: DecodeStep, reps: int):
-    """Average device duration of the document-pass kernel, from CUDA events
-    the library records around it on the launching stream, over `reps`
-    eager passes of all layers."""
+    """Average device duration of the document-pass kernel and of the suffix
+    kernel, from CUDA events the library records around them on the
+    launching stream.  The step with the events is captured as its own CUDA
+    graph (event-record nodes), so host launch overhead cannot leak into the
+    intervals; each replay re-records all 3 events of every layer."""
     pp = step.pp
-    opt = pp.Options()
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(step.layers)]
+    opts = []
+    for l in range(step.layers):
+        o = pp.Options()
+        o.set_events(evs[l])
+        opts.append(o)
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream(step.device)
+    s.wait_stream(torch.cuda.current_stream(step.device))
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            step.run_eager(opts=opts)
+    torch.cuda.current_stream(step.device).wait_stream(s)
     durs = {"doc": [], "suffix": []}
-    for _ in range(reps):
-        step.run_eager(opt=opt, layer_events=evs)
+    for _ in range(reps + 1):
+        g.replay()
         torch.cuda.synchronize()
         for e in evs:
             durs["doc"].append(e[0].elapsed_time(e[1]))
             durs["suffix"].append(e[1].elapsed_time(e[2]))
-    return {k: float(np.mean(v)) for k, v in durs.items()}
+    n = step.layers
+    del g
+    return {k: float(np.mean(v[n:])) for k, v in durs.items()}   # first replay = warm-up
 
 
 # ------------------------------------------------------------ CPU oracle ---

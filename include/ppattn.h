@@ -110,7 +110,9 @@ typedef struct pp_kv_layer {
  *                           decode/prefill record on `stream` before the
  *                           document pass, after it, and after the suffix
  *                           pass with its merge (per-kernel timing with CUDA
- *                           events; the work done is unchanged).
+ *                           events; the work done is unchanged).  During a
+ *                           stream capture they are recorded as external
+ *                           event-record nodes, i.e. at every graph replay.
  */
 typedef struct pp_options {
     int32_t splits;

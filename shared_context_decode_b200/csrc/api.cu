@@ -139,7 +139,16 @@ pp_status attend(const pp_kv_layer* L, int32_t doc_len, const uint16_t* q, const
   const Partials part = carve(ws, w);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaEvent_t* ev = (opt && opt->events) ? reinterpret_cast<cudaEvent_t*>(opt->events) : nullptr;
-  auto mark = [&](int i) { return ev ? cudaEventRecord(ev[i], st) : cudaSuccess; };
+  // Inside a stream capture the events become event-record nodes of the graph
+  // (recorded at every replay), so per-kernel timing also works for graphs.
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  if (ev && cudaStreamIsCapturing(st, &cap) != cudaSuccess) return PP_ERR_CUDA;
+  auto mark = [&](int i) {
+    if (!ev) return cudaSuccess;
+    return cap == cudaStreamCaptureStatusActive
+               ? cudaEventRecordWithFlags(ev[i], st, cudaEventRecordExternal)
+               : cudaEventRecord(ev[i], st);
+  };
   if (mark(0) != cudaSuccess) return PP_ERR_CUDA;
   if (has_doc) {
     cudaError_t e;

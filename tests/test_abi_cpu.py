@@ -109,7 +109,7 @@ def test_workspace_sizes_with_explicit_split(pp):
     (200, 4, 1000, 3), (300, 2, 300, 7), (1, 1, 1, 148), (256, 32, 16384, 1), (130, 3, 129, 5)])
 def test_split_plan_invariants(pp, rows, H, doc_len, ctas):
     p = pp.split_plan(rows, H, doc_len, ctas)
-    T = -(-doc_len // 128)
+    T = -(-doc_len // 128)       # document tile: 128 keys
     units = -(-rows // 256) * H
     assert p["T"] == T and p["units"] == units and p["W"] == units * T
     assert p["C"] == min(ctas, units * T)

@@ -34,7 +34,7 @@ def test_tiny_config_full():
     decode_case(wl.make_decode("tiny", device=DEV))
 
 
-@pytest.mark.parametrize("splits", [0, 1, 3, 7])
+@pytest.mark.parametrize("splits", [0, 1, 3, 5, 7, 16])
 def test_ragged_two_mtiles_split_variants(splits):
     # 8 key tiles with a 104-key tail, 200 rows = 128 + 72, 4 heads
     W = wl.make_decode(layers=1, H=4, d=128, N=1000, P=200, q=(1, 20), a=(0, 10), seed=1,
