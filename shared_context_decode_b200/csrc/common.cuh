@@ -130,7 +130,8 @@ __device__ __forceinline__ float2 ex2_poly2(float2 x) {
 
 // ---------------------------------------------------------------------------
 // Split plan of the document pass.  Work is the linear range of
-// units * T tiles, unit u = group * H + head, T = ceil(doc_len / kBN).  CTA c
+// units * T tiles, unit u = head * groups + group (head-major, so CTAs that
+// run at the same time share a head's K/V in L2), T = ceil(doc_len / kBN).  CTA c
 // owns tiles [floor(c*W/C), floor((c+1)*W/C)); every (unit, CTA) overlap is a
 // "chunk" with its own partial result slot u * max_chunks + (c - first CTA of
 // u).  Host and device evaluate the same integer formulas.
@@ -138,7 +139,7 @@ struct SplitPlan {
   int64_t W;        // total tiles
   int32_t C;        // CTAs
   int32_t T;        // tiles per unit
-  int32_t units;    // groups * H
+  int32_t units;    // H * groups
   int32_t max_chunks;
 };
 

@@ -10,10 +10,11 @@
 //     O += P V_tile           (M = 128, N = d, K = kBN; P bf16 read from TMEM)
 // Up to 256 query rows (two M tiles) share every K/V tile a CTA loads.
 //
-// Work split: the (row group, head, tile) space is cut into contiguous tile
-// ranges, one per persistent CTA (see SplitPlan); a CTA whose range crosses
-// into another head starts a new "segment" and writes one partial result per
-// segment.  The merge kernel combines the partials with the suffix pass.
+// Work split: the (head, row group, tile) space is cut into contiguous tile
+// ranges, one per persistent CTA (see SplitPlan; head-major, so CTAs running
+// at the same time share a head's K/V in L2); a CTA whose range crosses into
+// another unit starts a new "segment" and writes one partial result per
+// segment.  The suffix kernel's epilogue merges the partials.
 //
 // Warp roles (384 threads):
 //   warp 0       Q and K producer (TMA, 128-byte swizzle)
@@ -47,6 +48,7 @@ static_assert(128 * kRegsLow + 256 * kRegsHigh <= 384 * kRegsLaunch, "register s
 struct DocTcParams {
   int rows;
   int H;
+  int G;        // row groups of kGroupRows
   int doc_len;
   SplitPlan plan;
   float sl2;
@@ -106,8 +108,8 @@ __device__ __forceinline__ bool next_seg(const DocTcParams& p, int64_t& t, int64
   s.j0 = (int)(t - (int64_t)s.u * T);
   const int64_t ue = (int64_t)s.u * T + T;
   s.j1 = (int)((ue < t_end ? ue : t_end) - (int64_t)s.u * T);
-  s.g = s.u / p.H;
-  s.h = s.u - s.g * p.H;
+  s.h = s.u / p.G;   // unit u = head * G + group (head-major)
+  s.g = s.u - s.h * p.G;
   s.chunk = cta - plan_cta_of(p.plan, (int64_t)s.u * T);
   const int rows_g = min(kGroupRows, p.rows - s.g * kGroupRows);
   s.nm = rows_g > 128 ? 2 : 1;
@@ -555,10 +557,12 @@ EncodeTiledFn get_encode() {
   return fn;
 }
 
+}  // namespace
+
 // 3-D bf16 tensor map, 128-byte swizzle, out-of-range elements read as zero.
-bool make_map(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
-              uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t b0, uint32_t b1,
-              uint32_t b2) {
+bool make_tmap_bf16_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+                       uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t b0, uint32_t b1,
+                       uint32_t b2) {
   EncodeTiledFn enc = get_encode();
   if (!enc) return false;
   const cuuint64_t dims[3] = {d0, d1, d2};
@@ -571,16 +575,18 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+namespace {
+
 template <int D>
 cudaError_t launch_impl(const pp_kv_layer& L, int doc_len, const uint16_t* q, int rows, float scale,
                         const SplitPlan& plan, const Partials& part, long long wait_limit,
                         int inject, cudaStream_t st) {
   using C = DocCfg<D>;
   CUtensorMap mQ, mK, mV;
-  if (!make_map(&mQ, q, D, L.H, rows, (uint64_t)D * 2, (uint64_t)L.H * D * 2, 64, 1, 128) ||
-      !make_map(&mK, L.k_doc, D, doc_len, L.H, (uint64_t)D * 2, (uint64_t)L.doc_cap * D * 2, 64,
+  if (!make_tmap_bf16_3d(&mQ, q, D, L.H, rows, (uint64_t)D * 2, (uint64_t)L.H * D * 2, 64, 1, 128) ||
+      !make_tmap_bf16_3d(&mK, L.k_doc, D, doc_len, L.H, (uint64_t)D * 2, (uint64_t)L.doc_cap * D * 2, 64,
                 kBN, 1) ||
-      !make_map(&mV, L.v_doc, D, doc_len, L.H, (uint64_t)D * 2, (uint64_t)L.doc_cap * D * 2, 64,
+      !make_tmap_bf16_3d(&mV, L.v_doc, D, doc_len, L.H, (uint64_t)D * 2, (uint64_t)L.doc_cap * D * 2, 64,
                 kBN, 1))
     return cudaErrorInvalidValue;
   // Once per device: allow the dynamic shared memory, and check that the
@@ -604,6 +610,7 @@ cudaError_t launch_impl(const pp_kv_layer& L, int doc_len, const uint16_t* q, in
   DocTcParams prm;
   prm.rows = rows;
   prm.H = L.H;
+  prm.G = (rows + kGroupRows - 1) / kGroupRows;
   prm.doc_len = doc_len;
   prm.plan = plan;
   prm.sl2 = scale * kLog2e;

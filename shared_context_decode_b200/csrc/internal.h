@@ -1,6 +1,7 @@
 // Internal launchers of libppattn (not part of the C ABI).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -10,6 +11,12 @@ namespace pp {
 
 struct SplitPlan;
 struct Partials;
+
+// 3-D bf16 TMA tensor map with 128-byte swizzle (zero fill out of range);
+// dims innermost first, strides of dims 1 and 2 in bytes.
+bool make_tmap_bf16_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+                       uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t b0, uint32_t b1,
+                       uint32_t b2);
 
 cudaError_t launch_kv_append(const pp_kv_layer& L, const uint16_t* k, const uint16_t* v,
                              const int16_t* sid, const int32_t* pos, int n, cudaStream_t st);

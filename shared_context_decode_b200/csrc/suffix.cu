@@ -6,14 +6,18 @@
 // than the query).  The decode step (one row per stream) and the question
 // prefill (rows causal within their question) run the same kernel.
 //
-// Work item = (query row, head).  Segment (s-1, h) is S_cap contiguous rows of
-// d bf16 ([P_max][H][S_cap][d]), so an item's keys stream as one contiguous
-// block.  Every warp owns a ring of NS shared-memory stages; lane 0 fills them
-// with 1-D TMA bulk copies (CK keys of K and of V per stage) running NS-1
-// chunks ahead of the warp, across item boundaries, so HBM reads overlap the
-// arithmetic without holding the data in registers.  d/8 lanes share a key
-// (16 bytes each), scores are reduced with warp shuffles, softmax is online in
-// the log2 domain.
+// Work item = (query row, head).  Each warp owns a contiguous, balanced block
+// of items and a ring of NS shared-memory stages; lane 0 fills them with 1-D
+// bulk copies of exactly the live keys of a chunk (a segment's rows are
+// contiguous), NS-1 chunks ahead of the warp and across item boundaries.
+//
+// Scores: 8 lanes per key, each lane a 16-byte group g of every 128 bytes of
+// the row, so the 8 lanes of a shared-memory phase read one contiguous
+// 128-byte span; four passes cover the chunk's 16 keys and a butterfly
+// transpose-reduce leaves key 4 * (2 b2 + b1) + sub on lane (sub, b2, b1, *)
+// (lane = 8 sub + 4 b2 + 2 b1 + b0).  P V: lane j owns output dimensions
+// [j d/32, (j+1) d/32) and takes each key's probability by shuffle.  Online
+// softmax in the log2 domain.
 //
 // Epilogue (merge): the item's suffix partial is combined with the document
 // pass's partials of the same (row, head):
@@ -31,18 +35,18 @@ namespace pp {
 
 template <int D>
 struct SufCfg {
-  static constexpr int LPK = D / 8;        // lanes per key (16 bytes each)
-  static constexpr int KPI = 32 / LPK;     // keys a warp covers per step
-  static constexpr int CK = 16;            // keys per chunk
-  static constexpr int ROW = D * 2;        // bytes per key row
-  static constexpr int HALF = CK * ROW;    // K (or V) part of a stage
+  static constexpr int CK = 16;              // keys per chunk
+  static constexpr int ROWB = D * 2;         // bytes of one key row
+  static constexpr int HALF = CK * ROWB;     // K (or V) part of a stage
   static constexpr int STAGE = 2 * HALF;
-  static constexpr int NS = 3;             // stages per warp (NS-1 chunks in flight)
-  static constexpr int WARPS = 8;          // warps per CTA
-  static constexpr int TBL = 256;          // item-table entries per warp and round
-  static constexpr int PRE = 4;            // document partials prefetched per key group
+  static constexpr int NS = 2;               // stages per warp (NS-1 chunks in flight)
+  static constexpr int WARPS = 12;           // warps per CTA
+  static constexpr int TBL = 128;            // item-table entries per warp and round
+  static constexpr int PRE = 4;              // document partials prefetched per lane
+  static constexpr int G = D / 64;           // 16-byte groups per lane and key row
+  static constexpr int E = D / 32;           // output dims per lane
   static constexpr int SMEM = WARPS * NS * STAGE + WARPS * TBL * 16 + 128;
-  static_assert(CK % KPI == 0, "chunk covers whole warp steps");
+  static_assert(SMEM <= 227 * 1024, "dynamic shared memory above the per-CTA limit");
 };
 
 struct SufParams {
@@ -67,9 +71,9 @@ struct SufParams {
 };
 
 // Per-item record of the warp's table: stream id (0 when the row is not an
-// answer-stream query), query position, visible-segment length.
+// answer-stream query), query position, visible-segment length, raw stream id.
 struct ItemRec {
-  int s, qp, n, pad;
+  int s, qp, n, raw;
 };
 
 // Online-softmax state fold: (m, l, a) <- (m, l, a) (+) (m2, l2, a2).
@@ -119,6 +123,9 @@ __device__ __forceinline__ bool stage_wait(uint64_t* bar, uint32_t parity, volat
   }
 }
 
+// Lane holding the score of chunk key kk after the transpose-reduce.
+__device__ __forceinline__ int key_lane(int kk) { return (kk & 3) * 8 + (kk >> 2) * 2; }
+
 template <int D>
 __global__ void __launch_bounds__(SufCfg<D>::WARPS * 32) suffix_merge(const SufParams p) {
   using C = SufCfg<D>;
@@ -128,7 +135,9 @@ __global__ void __launch_bounds__(SufCfg<D>::WARPS * 32) suffix_merge(const SufP
   __shared__ uint64_t bars[C::WARPS][C::NS];
   __shared__ int abort_sh;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int g = lane / C::LPK, j = lane % C::LPK;
+  const int g = lane & 7, sub = lane >> 3;          // score: 16-byte group, key of a pass
+  const int b2 = (lane >> 2) & 1, b1 = (lane >> 1) & 1;
+  const int my_key = 4 * (2 * b2 + b1) + sub;       // key whose score this lane ends with
   uint8_t* ring = smem + warp * C::NS * C::STAGE;
   ItemRec* tbl = reinterpret_cast<ItemRec*>(smem + C::WARPS * C::NS * C::STAGE) + warp * C::TBL;
   uint64_t* full = bars[warp];
@@ -140,12 +149,13 @@ __global__ void __launch_bounds__(SufCfg<D>::WARPS * 32) suffix_merge(const SufP
   __syncthreads();
   volatile int* abort_flag = &abort_sh;
 
-  // This warp's items: a contiguous, balanced block of the (head, row) space
-  // (head-major, so in a prefill neighbouring items share a segment).
+  // This warp's items: a contiguous, balanced block of the (head, row) space,
+  // head-major, so in a prefill neighbouring items share a segment.
   const int64_t items = (int64_t)p.rows * p.H;
   const int64_t gw = (int64_t)blockIdx.x * C::WARPS + warp;
   const int64_t GW = (int64_t)gridDim.x * C::WARPS;
   const int64_t i_begin = gw * items / GW, i_end = (gw + 1) * items / GW;
+  const int groups = (p.rows + kGroupRows - 1) / kGroupRows;
   const size_t seg_elems = (size_t)p.S_cap * D;
 
   uint32_t issued = 0, consumed = 0;
@@ -155,14 +165,13 @@ __global__ void __launch_bounds__(SufCfg<D>::WARPS * 32) suffix_merge(const SufP
     // ---- item table of this round: two parallel gathers instead of one
     // dependent chain per item
     for (int k = lane; k < cnt; k += 32) {
-      const int64_t item = r0 + k;
-      const int r = (int)(item % p.rows);
+      const int r = (int)((r0 + k) % p.rows);
       const int s = p.q_sid[r];
       ItemRec rec;
       rec.qp = p.q_pos[r];
       rec.s = stream_query(s, p.P_max) ? s : 0;
       rec.n = 0;
-      rec.pad = s;
+      rec.raw = s;
       tbl[k] = rec;
     }
     __syncwarp();
@@ -186,13 +195,13 @@ __global__ void __launch_bounds__(SufCfg<D>::WARPS * 32) suffix_merge(const SufP
       if (lane == 0) {
         const ItemRec rec = tbl[pk];
         const int h = (int)((r0 + pk) / p.rows);
+        const size_t seg = ((size_t)(rec.s - 1) * p.H + h) * seg_elems + (size_t)pt0 * D;
         const int nk = min(C::CK, rec.n - pt0);
-        const size_t off = ((size_t)(rec.s - 1) * p.H + h) * seg_elems + (size_t)pt0 * D;
         uint8_t* st = ring + stage * C::STAGE;
         fence_proxy_async();
-        mbar_arrive_expect_tx(full + stage, 2u * nk * C::ROW);
-        bulk_load(st, p.k_suf + off, nk * C::ROW, full + stage);
-        bulk_load(st + C::HALF, p.v_suf + off, nk * C::ROW, full + stage);
+        mbar_arrive_expect_tx(full + stage, 2u * nk * C::ROWB);
+        bulk_load(st, p.k_suf + seg, nk * C::ROWB, full + stage);
+        bulk_load(st + C::HALF, p.v_suf + seg, nk * C::ROWB, full + stage);
       }
       pt0 += C::CK;
       return true;
@@ -205,54 +214,70 @@ __global__ void __launch_bounds__(SufCfg<D>::WARPS * 32) suffix_merge(const SufP
       const int h = (int)(item / p.rows), r = (int)(item - (int64_t)h * p.rows);
       const ItemRec rec = tbl[k];
       const bool valid = rec.s != 0;
-      // query fragment, and the document partials of this (row, head), fetched now
-      // so their latency hides behind the segment's chunks
-      const uint4 qv = reinterpret_cast<const uint4*>(p.q + ((int64_t)r * p.H + h) * D)[j];
+      // document partials of this (row, head), fetched now so their latency
+      // hides behind the segment's chunks
       int c0 = 0, c1 = -1;
       int64_t slot0 = 0;
       const int rr = r % kGroupRows;
       if (valid && p.has_doc) {
-        const int u = (r / kGroupRows) * p.H + h;
+        const int u = h * groups + r / kGroupRows;
         c0 = plan_cta_of(p.plan, (int64_t)u * p.plan.T);
         c1 = plan_cta_of(p.plan, (int64_t)u * p.plan.T + p.plan.T - 1);
         slot0 = (int64_t)u * p.plan.max_chunks;
       }
       float2 pre_ml[C::PRE];
-      float4 pre_o[C::PRE][2];
+      float pre_o[C::PRE][C::E];
 #pragma unroll
       for (int e = 0; e < C::PRE; ++e) {
-        const int c = c0 + g + e * C::KPI;
-        if (c <= c1) {
-          const int64_t sl = (slot0 + c - c0) * kGroupRows + rr;
+        if (c0 + e <= c1) {
+          const int64_t sl = (slot0 + e) * kGroupRows + rr;
           pre_ml[e] = *reinterpret_cast<const float2*>(p.doc_ml + sl * 2);
-          const float4* src = reinterpret_cast<const float4*>(p.doc_o + sl * D + j * 8);
-          pre_o[e][0] = src[0];
-          pre_o[e][1] = src[1];
+          const float* src = p.doc_o + sl * D + lane * C::E;
+          if (C::E == 4) {
+            const float4 v = *reinterpret_cast<const float4*>(src);
+            pre_o[e][0] = v.x; pre_o[e][1 % C::E] = v.y;
+            pre_o[e][2 % C::E] = v.z; pre_o[e][3 % C::E] = v.w;
+          } else {
+            const float2 v = *reinterpret_cast<const float2*>(src);
+            pre_o[e][0] = v.x; pre_o[e][1 % C::E] = v.y;
+          }
         }
       }
-      float qf[8];
+      // this lane's query dims (groups g, g + 8, ...), scaled by scale * log2(e)
+      float2 q2[C::G * 4];
       {
-        const uint32_t w[4] = {qv.x, qv.y, qv.z, qv.w};
+        const uint4* qp4 = reinterpret_cast<const uint4*>(p.q + ((int64_t)r * p.H + h) * D);
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const float2 f = bf2_to_f2(w[c]);
-          qf[2 * c] = f.x * p.sl2;
-          qf[2 * c + 1] = f.y * p.sl2;
+        for (int c = 0; c < C::G; ++c) {
+          const uint4 w = qp4[g + 8 * c];
+          const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float2 f = bf2_to_f2(ww[i]);
+            q2[c * 4 + i] = make_float2(f.x * p.sl2, f.y * p.sl2);
+          }
         }
       }
-      float m = -INFINITY, l = 0.f, acc[8];
+      float m = -INFINITY, lp = 0.f, acc[C::E];
 #pragma unroll
-      for (int c = 0; c < 8; ++c) acc[c] = 0.f;
+      for (int e = 0; e < C::E; ++e) acc[e] = 0.f;
       const int16_t* sb = p.sid + (size_t)(valid ? rec.s - 1 : 0) * p.S_cap;
       const int32_t* pb = p.pos + (size_t)(valid ? rec.s - 1 : 0) * p.S_cap;
 
+      // this lane's key tags, loaded one chunk ahead of their use
+      int nsid = -1, npos = 0;
+      if (my_key < rec.n) {
+        nsid = __ldg(sb + my_key);
+        npos = __ldg(pb + my_key);
+      }
       for (int t0 = 0; t0 < rec.n; t0 += C::CK) {
         if (issue_next(issued % C::NS)) ++issued;
-        const int nk = min(C::CK, rec.n - t0);
-        int tsid = -1, tpos = 0;  // this chunk's tags, one per lane (loaded before the wait)
-        if (lane < nk) {
-          tsid = __ldg(sb + t0 + lane);
-          tpos = __ldg(pb + t0 + lane);
+        const int t = t0 + my_key;
+        const int tsid = nsid, tpos = npos;
+        nsid = -1;
+        if (t + C::CK < rec.n) {
+          nsid = __ldg(sb + t + C::CK);
+          npos = __ldg(pb + t + C::CK);
         }
         const uint32_t stage = consumed % C::NS;
         if (!(ok = stage_wait(full + stage, (consumed / C::NS) & 1, abort_flag, p.wait_limit,
@@ -260,49 +285,73 @@ __global__ void __launch_bounds__(SufCfg<D>::WARPS * 32) suffix_merge(const SufP
           break;
         const uint8_t* sK = ring + stage * C::STAGE;
         const uint8_t* sV = sK + C::HALF;
-        float x[C::CK / C::KPI];
+        // partial dots of keys 4 j + sub (pass j) over this lane's groups;
+        // rows past the chunk's live keys hold stale bytes and are masked below
+        float v[4];
 #pragma unroll
-        for (int u = 0; u < C::CK / C::KPI; ++u) {
-          const int kk = u * C::KPI + g;
-          const uint4 kv = *reinterpret_cast<const uint4*>(sK + kk * C::ROW + j * 16);
-          const uint32_t w[4] = {kv.x, kv.y, kv.z, kv.w};
-          float dot = 0.f;
+        for (int j = 0; j < 4; ++j) {
+          const uint8_t* rowp = sK + (4 * j + sub) * C::ROWB + g * 16;
+          float2 d0 = make_float2(0.f, 0.f), d1 = make_float2(0.f, 0.f);
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            const float2 f = bf2_to_f2(w[c]);
-            dot = fmaf(qf[2 * c], f.x, dot);
-            dot = fmaf(qf[2 * c + 1], f.y, dot);
+          for (int c = 0; c < C::G; ++c) {
+            const uint4 w = *reinterpret_cast<const uint4*>(rowp + c * 128);
+            d0 = ffma2(q2[c * 4 + 0], bf2_to_f2(w.x), d0);
+            d1 = ffma2(q2[c * 4 + 1], bf2_to_f2(w.y), d1);
+            d0 = ffma2(q2[c * 4 + 2], bf2_to_f2(w.z), d0);
+            d1 = ffma2(q2[c * 4 + 3], bf2_to_f2(w.w), d1);
+          }
+          v[j] = (d0.x + d0.y) + (d1.x + d1.y);
+        }
+        // this lane's V words of every key of the chunk, loaded while the
+        // score reduction runs (d/32 bf16 values per key)
+        uint32_t vw[C::CK][C::E / 2];
+#pragma unroll
+        for (int kk = 0; kk < C::CK; ++kk) {
+          if (C::E == 4) {
+            const uint2 w = *reinterpret_cast<const uint2*>(sV + kk * C::ROWB + lane * 8);
+            vw[kk][0] = w.x;
+            vw[kk][1 % (C::E / 2)] = w.y;
+          } else {
+            vw[kk][0] = *reinterpret_cast<const uint32_t*>(sV + kk * C::ROWB + lane * 4);
+          }
+        }
+        // transpose-reduce over the 8 lanes of a key group: xor 4 splits the
+        // passes {0,1} | {2,3}, xor 2 splits the pair, xor 1 finishes the sum
+        float w0, w1;
+        {
+          const float r0s = __shfl_xor_sync(0xffffffffu, b2 ? v[0] : v[2], 4);
+          const float r1s = __shfl_xor_sync(0xffffffffu, b2 ? v[1] : v[3], 4);
+          w0 = (b2 ? v[2] : v[0]) + r0s;
+          w1 = (b2 ? v[3] : v[1]) + r1s;
+        }
+        float dot = (b1 ? w1 : w0) + __shfl_xor_sync(0xffffffffu, b1 ? w0 : w1, 2);
+        dot += __shfl_xor_sync(0xffffffffu, dot, 1);
+        const float x = slot_visible(rec.s, rec.qp, tsid, tpos, t, rec.n) ? dot : -INFINITY;
+        float cm = fmaxf(m, x);
+#pragma unroll
+        for (int o = 2; o < 32; o <<= 1) cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, o));
+        if (cm != -INFINITY) {  // warp-uniform
+          const float corr = exp2f(m - cm);  // m = -inf gives 0
+          const float pr = exp2f(x - cm);    // masked keys give 0
+          lp = lp * corr + ((lane & 1) ? 0.f : pr);
+          const uint32_t live = __ballot_sync(0xffffffffu, pr > 0.f);
+          float2 a2[C::E / 2];
+#pragma unroll
+          for (int e = 0; e < C::E / 2; ++e) a2[e] = make_float2(acc[2 * e] * corr, acc[2 * e + 1] * corr);
+          // P V: a dead key's V words are zeroed, not weighted by 0 (rows past
+          // a segment's end hold stale data)
+#pragma unroll
+          for (int kk = 0; kk < C::CK; ++kk) {
+            const float pk = __shfl_sync(0xffffffffu, pr, key_lane(kk));
+            const bool on = (live >> key_lane(kk)) & 1u;
+            const float2 pk2 = make_float2(pk, pk);
+#pragma unroll
+            for (int e = 0; e < C::E / 2; ++e) a2[e] = ffma2(pk2, bf2_to_f2(on ? vw[kk][e] : 0u), a2[e]);
           }
 #pragma unroll
-          for (int o = 1; o < C::LPK; o <<= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
-          const int ks = __shfl_sync(0xffffffffu, tsid, kk);
-          const int kp = __shfl_sync(0xffffffffu, tpos, kk);
-          x[u] = (kk < nk && slot_visible(rec.s, rec.qp, ks, kp, t0 + kk, rec.n)) ? dot : -INFINITY;
-        }
-        float cm = m;
-#pragma unroll
-        for (int u = 0; u < C::CK / C::KPI; ++u) cm = fmaxf(cm, x[u]);
-        if (cm != -INFINITY) {
-          const float corr = exp2f(m - cm);
-          l *= corr;
-#pragma unroll
-          for (int c = 0; c < 8; ++c) acc[c] *= corr;
-#pragma unroll
-          for (int u = 0; u < C::CK / C::KPI; ++u) {
-            // masked keys are skipped, not weighted by 0: stage rows past the
-            // chunk's end hold stale shared memory
-            if (x[u] == -INFINITY) continue;
-            const float pr = exp2f(x[u] - cm);
-            l += pr;
-            const int kk = u * C::KPI + g;
-            const uint4 vv = *reinterpret_cast<const uint4*>(sV + kk * C::ROW + j * 16);
-            const uint32_t w[4] = {vv.x, vv.y, vv.z, vv.w};
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              const float2 f = bf2_to_f2(w[c]);
-              acc[2 * c] = fmaf(pr, f.x, acc[2 * c]);
-              acc[2 * c + 1] = fmaf(pr, f.y, acc[2 * c + 1]);
-            }
+          for (int e = 0; e < C::E / 2; ++e) {
+            acc[2 * e] = a2[e].x;
+            acc[2 * e + 1] = a2[e].y;
           }
           m = cm;
         }
@@ -312,43 +361,43 @@ __global__ void __launch_bounds__(SufCfg<D>::WARPS * 32) suffix_merge(const SufP
       if (!ok) break;
 
       // ---- merge with the document partials of (row, head)
-      combine_groups<C::LPK>(m, l, acc);
-      if (g != 0) {  // group 0 carries the suffix partial, the others start empty
-        m = -INFINITY;
-        l = 0.f;
+      float l = lp;
 #pragma unroll
-        for (int c = 0; c < 8; ++c) acc[c] = 0.f;
-      }
+      for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+      auto fold_in = [&](float m2, float l2, const float* a2) {
+        const float mm = fmaxf(m, m2);
+        const float xa = (m == -INFINITY) ? 0.f : exp2f(m - mm);
+        const float ya = (m2 == -INFINITY) ? 0.f : exp2f(m2 - mm);
+        l = l * xa + l2 * ya;
 #pragma unroll
-      for (int e = 0; e < C::PRE; ++e) {
-        if (c0 + g + e * C::KPI <= c1) {
-          const float a2[8] = {pre_o[e][0].x, pre_o[e][0].y, pre_o[e][0].z, pre_o[e][0].w,
-                               pre_o[e][1].x, pre_o[e][1].y, pre_o[e][1].z, pre_o[e][1].w};
-          fold(m, l, acc, pre_ml[e].x, pre_ml[e].y, a2);
-        }
-      }
-      for (int c = c0 + g + C::PRE * C::KPI; c <= c1; c += C::KPI) {
+        for (int e = 0; e < C::E; ++e) acc[e] = acc[e] * xa + a2[e] * ya;
+        m = mm;
+      };
+#pragma unroll
+      for (int e = 0; e < C::PRE; ++e)
+        if (c0 + e <= c1) fold_in(pre_ml[e].x, pre_ml[e].y, pre_o[e]);
+      for (int c = c0 + C::PRE; c <= c1; ++c) {
         const int64_t sl = (slot0 + c - c0) * kGroupRows + rr;
         const float2 ml = *reinterpret_cast<const float2*>(p.doc_ml + sl * 2);
-        const float4* src = reinterpret_cast<const float4*>(p.doc_o + sl * D + j * 8);
-        const float4 a0 = src[0], a1 = src[1];
-        const float a2[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-        fold(m, l, acc, ml.x, ml.y, a2);
+        float a2[C::E];
+#pragma unroll
+        for (int e = 0; e < C::E; ++e) a2[e] = p.doc_o[sl * D + lane * C::E + e];
+        fold_in(ml.x, ml.y, a2);
       }
-      combine_groups<C::LPK>(m, l, acc);
       const bool any = valid && l > 0.f;
       const float inv = any ? 1.f / l : 0.f;
-      if (g == 0) {
-        uint4 pkd;
-        pkd.x = f2_to_bf2(acc[0] * inv, acc[1] * inv);
-        pkd.y = f2_to_bf2(acc[2] * inv, acc[3] * inv);
-        pkd.z = f2_to_bf2(acc[4] * inv, acc[5] * inv);
-        pkd.w = f2_to_bf2(acc[6] * inv, acc[7] * inv);
-        reinterpret_cast<uint4*>(p.o + ((int64_t)r * p.H + h) * D)[j] = pkd;
+      uint16_t* dst = p.o + ((int64_t)r * p.H + h) * D + lane * C::E;
+      if (C::E == 4) {
+        uint2 pkd;
+        pkd.x = f2_to_bf2(acc[0] * inv, acc[1 % C::E] * inv);
+        pkd.y = f2_to_bf2(acc[2 % C::E] * inv, acc[3 % C::E] * inv);
+        *reinterpret_cast<uint2*>(dst) = pkd;
+      } else {
+        *reinterpret_cast<uint32_t*>(dst) = f2_to_bf2(acc[0] * inv, acc[1 % C::E] * inv);
       }
       if (lane == 0) {
         if (p.lse) p.lse[(int64_t)r * p.H + h] = any ? (m + log2f(l)) * kLn2 : -INFINITY;
-        if (h == 0 && (rec.pad == 0 || rec.pad > p.P_max)) set_status(p.status, PP_DEV_BAD_STREAM);
+        if (h == 0 && (rec.raw == 0 || rec.raw > p.P_max)) set_status(p.status, PP_DEV_BAD_STREAM);
       }
     }
     __syncwarp();
@@ -412,7 +461,7 @@ cudaError_t launch_suffix_merge(const pp_kv_layer& L, const uint16_t* q, const i
 // head) over all doc_len keys, no tensor cores.  This is what serving each
 // question as its own request costs (the page's "Inside decode step":
 // batched requests read the document keys once per question).  Writes the
-// document partial of chunk 0 of unit (row / kGroupRows) * H + h, which the
+// document partial of chunk 0 of unit h * groups + row / kGroupRows, which the
 // suffix kernel's merge then finishes; the plan it pairs with has one chunk
 // per unit.
 template <int D>
@@ -493,7 +542,7 @@ __global__ void __launch_bounds__(256) doc_per_stream(pp_kv_layer L, int doc_len
     m = cm;
   }
   combine_groups<LPK>(m, l, acc);
-  const int64_t slot = ((int64_t)(r / kGroupRows) * L.H + h) * max_chunks;
+  const int64_t slot = ((int64_t)h * ((rows + kGroupRows - 1) / kGroupRows) + r / kGroupRows) * max_chunks;
   const int rr = r % kGroupRows;
   if (g == 0) {
     float4* dst = reinterpret_cast<float4*>(doc_o + (slot * kGroupRows + rr) * D + j * 8);
