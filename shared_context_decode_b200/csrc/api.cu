@@ -84,7 +84,9 @@ SplitPlan ablation_plan(int rows, int H, int doc_len) {
 
 SplitPlan plan_for(int rows, int H, int doc_len, const pp_options* opt) {
   if (opt && opt->ablation_doc_per_stream) return ablation_plan(rows, H, doc_len);
-  const int ctas = (opt && opt->splits > 0) ? opt->splits : sm_count();
+  // one slot (a CTA per M tile of a row group) per SM pair by default
+  const int ctas = (opt && opt->splits > 0) ? opt->splits
+                                           : std::max(1, sm_count() / pp::doc_pair_ctas(rows));
   return make_plan(rows, H, doc_len, ctas);
 }
 

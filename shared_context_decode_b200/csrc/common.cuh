@@ -23,6 +23,9 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 // Rows of queries one document-pass CTA stacks as the MMA M dimension.
 constexpr int kGroupRows = 256;
+// CTAs per document-pass slot: one per 128-row M tile of a row group, so two
+// as soon as some row group holds more than 128 rows.
+__host__ __device__ inline int doc_pair_ctas(int rows) { return rows > 128 ? 2 : 1; }
 // Keys per document tile (the N of S = Q K^T, the K of O = P V).
 constexpr int kBN = 128;
 
@@ -198,6 +201,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
       : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// As mbar_try_wait, but the thread may sleep until the phase completes or
+// about `ns` nanoseconds pass, so a waiting warp leaves the issue slots of
+// its sub-partition to the warps that have work.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(ns)
       : "memory");
   return ok != 0;
 }

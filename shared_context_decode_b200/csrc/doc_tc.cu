@@ -5,26 +5,31 @@
 // head are stacked into one matrix, so each decode step reads the document
 // keys once ("1 matrix x matrix product").  Here that matrix product is a
 // tcgen05 MMA with the queries as M: per head h and document tile of kBN keys,
-//     S = Q_h K_tile^T        (M = 128 query rows per tile, N = kBN, K = d)
+//     S = Q_h K_tile^T        (M = 128 query rows, N = kBN, K = d)
 //     online softmax of S in fp32 (log2 domain, lazily rescaled)
 //     O += P V_tile           (M = 128, N = d, K = kBN; P bf16 read from TMEM)
-// Up to 256 query rows (two M tiles) share every K/V tile a CTA loads.
 //
 // Work split: the (head, row group, tile) space is cut into contiguous tile
-// ranges, one per persistent CTA (see SplitPlan; head-major, so CTAs running
-// at the same time share a head's K/V in L2); a CTA whose range crosses into
-// another unit starts a new "segment" and writes one partial result per
-// segment.  The suffix kernel's epilogue merges the partials.
+// ranges, one per "slot" (see SplitPlan; head-major, so slots running at the
+// same time share a head's K/V in L2).  A row group is 256 query rows = two
+// M tiles; a slot is a pair of CTAs, one per M tile, launched next to each
+// other and walking the same tiles, so the second CTA's K/V reads hit L2.  A
+// slot whose range crosses into another unit starts a new "segment" and
+// writes one partial result per segment; the suffix kernel's epilogue merges
+// the partials.
 //
 // Warp roles (384 threads):
 //   warp 0       Q and K producer (TMA, 128-byte swizzle)
-//   warp 1       MMA issuer (one thread)
+//   warp 1       MMA issuer (warp-uniform, one elected lane issues)
 //   warp 2       TMEM allocator
 //   warp 3       V producer
-//   warps 4-7    softmax of M tile 0 (thread = query row = TMEM lane)
-//   warps 8-11   softmax of M tile 1
-// TMEM (512 columns): O0 | O1 | S0 | S1; P_i overwrites the first kBN/2
-// columns of S_i (bf16 pairs) once the softmax has read S_i.
+//   warps 4-11   softmax: warp w owns 32 rows (its TMEM lane quarter w % 4)
+//                and one half of the kBN columns; the two warps of a lane
+//                quarter swap their partial row maxima through shared memory
+// TMEM: O | S0 | S1.  The two S buffers alternate by tile, so the MMA warp
+// issues S_{j+2} = Q K_{j+2}^T right behind O += P_j V_j and the softmax of
+// tile j + 1 never waits for the product of tile j; P_j overwrites the first
+// kBN/2 columns of its S buffer once both halves have read it.
 //
 // Every wait is bounded: on expiry the kernel sets PP_DEV_TIMEOUT, raises a
 // CTA-wide abort flag, drains its own copies and MMAs (bounded), frees TMEM
@@ -42,13 +47,15 @@ namespace pp {
 // Register split: the block is launched with kRegsLaunch registers per thread
 // (384 * 168 = 64512); warps 0-3 drop to kRegsLow and the 8 softmax warps
 // rise to kRegsHigh, which adds up to exactly the launch total.
+constexpr int kThreads = 384;
 constexpr int kRegsLaunch = 168, kRegsLow = 88, kRegsHigh = 208;
-static_assert(128 * kRegsLow + 256 * kRegsHigh <= 384 * kRegsLaunch, "register split");
+static_assert(128 * kRegsLow + 256 * kRegsHigh <= kThreads * kRegsLaunch, "register split");
 
 struct DocTcParams {
   int rows;
   int H;
   int G;        // row groups of kGroupRows
+  int pair;     // CTAs per slot: 2 when some row group has two M tiles, else 1
   int doc_len;
   SplitPlan plan;
   float sl2;
@@ -63,22 +70,24 @@ template <int D>
 struct DocCfg {
   static constexpr int KH = D / 64;                  // 128-byte column halves of a row
   static constexpr int BOX = 128 * 64 * 2;           // one [128 x 64] bf16 TMA box
-  static constexpr int Q_BYTES = 2 * KH * BOX;       // two M tiles
+  static constexpr int Q_BYTES = KH * BOX;           // one M tile
   static constexpr int KV_STAGE = KH * BOX;          // one tile of kBN = 128 keys
-  static constexpr int NK = 2, NV = 2;
+  static constexpr int NK = 3, NV = 2;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + Q_BYTES;
   static constexpr int OFF_V = OFF_K + NK * KV_STAGE;
   static constexpr int OFF_BAR = OFF_V + NV * KV_STAGE;
   // q_full, q_empty, k_full[NK], k_empty[NK], v_full[NV], v_empty[NV],
-  // s_full[2], p_full[2], o_done[2], o_free[2], drain
-  static constexpr int NBAR = 2 + 2 * NK + 2 * NV + 8 + 1;
+  // s_full[2], p_full[2], pv_done, o_done, o_free, drain
+  static constexpr int NBAR = 2 + 2 * NK + 2 * NV + 8;
   static constexpr int USED = OFF_BAR + NBAR * 8;
   // +1 KB for 1024-byte alignment; at least 120 KB so one CTA owns an SM's TMEM.
   static constexpr int SMEM = (USED + 1024) > 120 * 1024 ? (USED + 1024) : 120 * 1024;
-  static constexpr uint32_t T_O0 = 0, T_O1 = D, T_S0 = 2 * D, T_S1 = 2 * D + kBN;
+  // the per-CTA limit covers the static exchange buffer (4 KB) as well
+  static_assert(SMEM + 4352 <= 227 * 1024, "shared memory above the per-CTA limit");
+  static constexpr uint32_t T_O = 0, T_S = D;        // S buffer b at T_S + b * kBN
   static constexpr uint32_t TMEM_COLS = 512;
-  static_assert(T_S1 + kBN <= TMEM_COLS, "TMEM budget");
+  static_assert(T_S + 2 * kBN <= TMEM_COLS, "TMEM budget");
   static_assert(kBN == 128, "one TMA box of keys per tile");
 };
 
@@ -89,19 +98,22 @@ struct Bars {
   uint64_t* k_empty;
   uint64_t* v_full;
   uint64_t* v_empty;
-  uint64_t* s_full;
-  uint64_t* p_full;
+  uint64_t* s_full;   // [b]
+  uint64_t* p_full;   // [b]
+  uint64_t* pv_done;
   uint64_t* o_done;
   uint64_t* o_free;
   uint64_t* drain;
 };
 
-// Segment iteration shared by every role.
+// Segment iteration shared by every role.  mt: this CTA's M tile of the
+// row group; active: the row group has rows in that M tile.
 struct Seg {
-  int u, g, h, j0, j1, chunk, nm;
+  int u, g, h, j0, j1, chunk;
+  bool active;
 };
-__device__ __forceinline__ bool next_seg(const DocTcParams& p, int64_t& t, int64_t t_end, int cta,
-                                         Seg& s) {
+__device__ __forceinline__ bool next_seg(const DocTcParams& p, int64_t& t, int64_t t_end, int slot,
+                                         int mt, Seg& s) {
   if (t >= t_end) return false;
   const int T = p.plan.T;
   s.u = (int)(t / T);
@@ -110,9 +122,8 @@ __device__ __forceinline__ bool next_seg(const DocTcParams& p, int64_t& t, int64
   s.j1 = (int)((ue < t_end ? ue : t_end) - (int64_t)s.u * T);
   s.h = s.u / p.G;   // unit u = head * G + group (head-major)
   s.g = s.u - s.h * p.G;
-  s.chunk = cta - plan_cta_of(p.plan, (int64_t)s.u * T);
-  const int rows_g = min(kGroupRows, p.rows - s.g * kGroupRows);
-  s.nm = rows_g > 128 ? 2 : 1;
+  s.chunk = slot - plan_cta_of(p.plan, (int64_t)s.u * T);
+  s.active = s.g * kGroupRows + mt * 128 < p.rows;
   t = (int64_t)s.u * T + s.j1;
   return true;
 }
@@ -123,7 +134,7 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
   const int lane = threadIdx.x & 31;
   const long long t0 = clock64();
   while (true) {
-    const bool ok = mbar_try_wait(bar, parity);
+    const bool ok = mbar_try_wait_sleep(bar, parity, 20000);
     if (__all_sync(0xffffffffu, ok)) return true;
     int stop = 0;
     if (lane == 0) {
@@ -145,7 +156,7 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
 __device__ __forceinline__ constexpr bool use_poly(int pair) { return pair % 5 == 1 || pair % 5 == 3; }
 
 template <int D>
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(kThreads, 1)
     doc_pass_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const DocTcParams p) {
   using C = DocCfg<D>;
@@ -154,6 +165,9 @@ __global__ void __launch_bounds__(384, 1)
                                              ~uintptr_t(1023));
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
+  // Lane-quarter exchange between the two column halves: [parity][half][row]
+  // = (sequence number << 32) | value bits.
+  __shared__ unsigned long long xch[2][2][128];
   volatile int* abort_flag = &abort_sh;
 
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
@@ -166,14 +180,16 @@ __global__ void __launch_bounds__(384, 1)
   B.v_empty = B.v_full + C::NV;
   B.s_full = B.v_empty + C::NV;
   B.p_full = B.s_full + 2;
-  B.o_done = B.p_full + 2;
-  B.o_free = B.o_done + 2;
-  B.drain = B.o_free + 2;
+  B.pv_done = B.p_full + 2;
+  B.o_done = B.pv_done + 1;
+  B.o_free = B.o_done + 1;
+  B.drain = B.o_free + 1;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int cta = blockIdx.x;
-  const int64_t t_begin = plan_tile_begin(p.plan, cta);
-  const int64_t t_end = plan_tile_begin(p.plan, cta + 1);
+  const int slot = blockIdx.x / p.pair;
+  const int mt = blockIdx.x - slot * p.pair;   // this CTA's M tile
+  const int64_t t_begin = plan_tile_begin(p.plan, slot);
+  const int64_t t_end = plan_tile_begin(p.plan, slot + 1);
 
   if (threadIdx.x == 0) {
     mbar_init(B.q_full, 1);
@@ -188,14 +204,16 @@ __global__ void __launch_bounds__(384, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(B.s_full + i, 1);
-      mbar_init(B.p_full + i, 128);
-      mbar_init(B.o_done + i, 1);
-      mbar_init(B.o_free + i, 128);
+      mbar_init(B.p_full + i, 256);
     }
+    mbar_init(B.pv_done, 1);
+    mbar_init(B.o_done, 1);
+    mbar_init(B.o_free, 256);
     mbar_init(B.drain, 1);
     abort_sh = 0;
-    fence_mbar_init();
   }
+  for (int i = threadIdx.x; i < 2 * 2 * 128; i += kThreads) (&xch[0][0][0])[i] = 0ull;
+  if (threadIdx.x == 0) fence_mbar_init();
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tmQ);
     prefetch_tmap(&tmK);
@@ -218,16 +236,16 @@ __global__ void __launch_bounds__(384, 1)
     Seg s;
     int kt = 0, nseg = 0;
     bool ok = true;
-    while (ok && next_seg(p, t, t_end, cta, s)) {
+    while (ok && next_seg(p, t, t_end, slot, mt, s)) {
+      if (!s.active) continue;
       if (nseg > 0 &&
           !(ok = warp_wait(B.q_empty, (nseg - 1) & 1, abort_flag, p.wait_limit, p.status)))
         break;
       if (elect_one()) {
-        mbar_arrive_expect_tx(B.q_full, s.nm * C::KH * C::BOX);
-        for (int mt = 0; mt < s.nm; ++mt)
-          for (int kh = 0; kh < C::KH; ++kh)
-            tma_load_3d(smem + C::OFF_Q + (mt * C::KH + kh) * C::BOX, &tmQ, B.q_full, kh * 64, s.h,
-                        s.g * kGroupRows + mt * 128);
+        mbar_arrive_expect_tx(B.q_full, C::KH * C::BOX);
+        for (int kh = 0; kh < C::KH; ++kh)
+          tma_load_3d(smem + C::OFF_Q + kh * C::BOX, &tmQ, B.q_full, kh * 64, s.h,
+                      s.g * kGroupRows + mt * 128);
       }
       for (int j = s.j0; j < s.j1; ++j, ++kt) {
         const int st = kt % C::NK, f = kt / C::NK;
@@ -260,7 +278,8 @@ __global__ void __launch_bounds__(384, 1)
     Seg s;
     int vt = 0;
     bool ok = true;
-    while (ok && next_seg(p, t, t_end, cta, s)) {
+    while (ok && next_seg(p, t, t_end, slot, mt, s)) {
+      if (!s.active) continue;
       for (int j = s.j0; j < s.j1; ++j, ++vt) {
         const int st = vt % C::NV, f = vt / C::NV;
         if (f > 0 &&
@@ -294,19 +313,18 @@ __global__ void __launch_bounds__(384, 1)
     const uint64_t dQ = smem_desc_sw128(smem_u32(smem + C::OFF_Q), 16, 1024);
     const uint64_t dK = smem_desc_sw128(smem_u32(smem + C::OFF_K), 16, 1024);
     const uint64_t dV = smem_desc_sw128(smem_u32(smem + C::OFF_V), C::BOX, 1024);
-    auto issue_qk = [&](int mt, int kslot) {
-      const uint32_t d_t = tmem + (mt ? C::T_S1 : C::T_S0);
-      const uint64_t a0 = dQ + (uint64_t)((mt * C::KH * C::BOX) >> 4);
+    auto issue_qk = [&](int b, int kslot) {
+      const uint32_t d_t = tmem + C::T_S + (uint32_t)(b * kBN);
       const uint64_t b0 = dK + (uint64_t)((kslot * C::KV_STAGE) >> 4);
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
         const uint64_t off = (uint64_t)(((kk >> 2) * C::BOX + (kk & 3) * 32) >> 4);
-        if (elect_one()) mma_ss(d_t, a0 + off, b0 + off, IDESC_QK, kk > 0 ? 1u : 0u);
+        if (elect_one()) mma_ss(d_t, dQ + off, b0 + off, IDESC_QK, kk > 0 ? 1u : 0u);
       }
     };
-    auto issue_pv = [&](int mt, int vslot, bool acc) {
-      const uint32_t d_t = tmem + (mt ? C::T_O1 : C::T_O0);
-      const uint32_t a_t = tmem + (mt ? C::T_S1 : C::T_S0);
+    auto issue_pv = [&](int b, int vslot, bool acc) {
+      const uint32_t d_t = tmem + C::T_O;
+      const uint32_t a_t = tmem + C::T_S + (uint32_t)(b * kBN);
       const uint64_t b0 = dV + (uint64_t)((vslot * C::KV_STAGE) >> 4);
 #pragma unroll
       for (int kk = 0; kk < kBN / 16; ++kk)
@@ -321,76 +339,59 @@ __global__ void __launch_bounds__(384, 1)
     int64_t t = t_begin;
     Seg s;
     int kt = 0, vt = 0, nseg = 0;
-    uint32_t pf_ph0 = 0, pf_ph1 = 0;
-    int used0 = 0, used1 = 0;  // segments in which each M tile has been active
+    uint32_t pf_ph = 0;   // bit b: parity of p_full[b]
     bool ok = true;
-    while (ok && next_seg(p, t, t_end, cta, s)) {
+    while (ok && next_seg(p, t, t_end, slot, mt, s)) {
+      if (!s.active) continue;
       if (!(ok = warp_wait(B.q_full, nseg & 1, abort_flag, p.wait_limit, p.status))) break;
-      if (!(ok = warp_wait(B.k_full + kt % C::NK, (kt / C::NK) & 1, abort_flag, p.wait_limit,
-                           p.status)))
-        break;
-      tc_fence_after();
-      issue_qk(0, kt % C::NK);
-      commit(B.s_full + 0);
-      if (s.nm > 1) {
-        issue_qk(1, kt % C::NK);
-        commit(B.s_full + 1);
+      const int n = s.j1 - s.j0;
+      // prologue: S_0 and S_1
+      for (int j = 0; ok && j < 2 && j < n; ++j) {
+        if (!(ok = warp_wait(B.k_full + kt % C::NK, (kt / C::NK) & 1, abort_flag, p.wait_limit,
+                             p.status)))
+          break;
+        tc_fence_after();
+        issue_qk(j, kt % C::NK);
+        commit(B.s_full + j);
+        commit(B.k_empty + kt % C::NK);
+        ++kt;
+        if (j == n - 1) commit(B.q_empty);
       }
-      commit(B.k_empty + kt % C::NK);
-      ++kt;
-      if (s.j1 - s.j0 == 1) commit(B.q_empty);
-      for (int j = s.j0; ok && j < s.j1; ++j) {
+      for (int j = 0; ok && j < n; ++j) {
+        const int b = j & 1;
         const int vslot = vt % C::NV;
         if (!(ok = warp_wait(B.v_full + vslot, (vt / C::NV) & 1, abort_flag, p.wait_limit, p.status)))
           break;
-        const bool has_next = j + 1 < s.j1;
-        const int kslot = kt % C::NK;
-        // ---- M tile 0
         // The first O += P V of a segment overwrites O: wait until the
-        // softmax has read out the previous segment that used this tile.
-        if (j == s.j0 && used0 > 0 &&
-            !(ok = warp_wait(B.o_free + 0, (used0 - 1) & 1, abort_flag, p.wait_limit, p.status)))
+        // softmax has read out the previous segment's O.
+        if (j == 0 && nseg > 0 &&
+            !(ok = warp_wait(B.o_free, (nseg - 1) & 1, abort_flag, p.wait_limit, p.status)))
           break;
-        if (!(ok = warp_wait(B.p_full + 0, pf_ph0, abort_flag, p.wait_limit, p.status))) break;
-        pf_ph0 ^= 1;
+        if (!(ok = warp_wait(B.p_full + b, (pf_ph >> b) & 1, abort_flag, p.wait_limit, p.status)))
+          break;
+        pf_ph ^= 1u << b;
         tc_fence_after();
-        issue_pv(0, vslot, j > s.j0);
-        if (has_next) {
+        issue_pv(b, vslot, j > 0);
+        commit(B.pv_done);
+        commit(B.v_empty + vslot);
+        ++vt;
+        if (j + 2 < n) {
+          // S_{j+2} reuses buffer b; the MMA pipe runs in issue order, so it
+          // is written only after this P V has read P_j.
+          const int kslot = kt % C::NK;
           if (!(ok = warp_wait(B.k_full + kslot, (kt / C::NK) & 1, abort_flag, p.wait_limit,
                                p.status)))
             break;
           tc_fence_after();
-          issue_qk(0, kslot);
-          commit(B.s_full + 0);
-        } else {
-          commit(B.o_done + 0);
-        }
-        // ---- M tile 1
-        if (s.nm > 1) {
-          if (j == s.j0 && used1 > 0 &&
-              !(ok = warp_wait(B.o_free + 1, (used1 - 1) & 1, abort_flag, p.wait_limit, p.status)))
-            break;
-          if (!(ok = warp_wait(B.p_full + 1, pf_ph1, abort_flag, p.wait_limit, p.status))) break;
-          pf_ph1 ^= 1;
-          tc_fence_after();
-          issue_pv(1, vslot, j > s.j0);
-          if (has_next) {
-            issue_qk(1, kslot);
-            commit(B.s_full + 1);
-          } else {
-            commit(B.o_done + 1);
-          }
-        }
-        commit(B.v_empty + vslot);
-        ++vt;
-        if (has_next) {
+          issue_qk(b, kslot);
+          commit(B.s_full + b);
           commit(B.k_empty + kslot);
           ++kt;
-          if (j + 2 == s.j1) commit(B.q_empty);
+          if (j + 3 == n) commit(B.q_empty);
+        } else if (j == n - 1) {
+          commit(B.o_done);
         }
       }
-      ++used0;
-      if (s.nm > 1) ++used1;
       ++nseg;
     }
     if (!ok) {
@@ -402,128 +403,171 @@ __global__ void __launch_bounds__(384, 1)
     }
   } else if (warp == 2) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLow));
-  } else if (warp >= 4) {
+  } else {
     // ---------------------------------------------------------- softmax ----
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsHigh));
-    const int wg = (warp - 4) >> 2;          // M tile
+    const int hf = (warp - 4) >> 2;          // column half
     const int wq = warp & 3;                 // TMEM lane quarter of this warp
     const int rt = wq * 32 + lane;           // row inside the M tile
+    constexpr int HB = kBN / 2;              // columns of S per half
+    constexpr int OC = D / 64;               // 32-column chunks of O per half
     const uint32_t t_lane = tmem + ((uint32_t)(wq * 32) << 16);
-    const uint32_t t_S = t_lane + (wg ? C::T_S1 : C::T_S0);
-    const uint32_t t_O = t_lane + (wg ? C::T_O1 : C::T_O0);
+    const uint32_t t_O = t_lane + C::T_O + hf * (D / 2);
     int64_t t = t_begin;
     Seg s;
-    uint32_t s_ph = 0, od_ph = 0;
+    uint32_t s_ph = 0, od_ph = 0;  // s_ph bit b: parity of s_full[b]
+    uint32_t g = 0;                // tiles so far = O += P V products issued before this one
+    uint32_t seq = 0;              // exchanges so far; both halves count alike
     bool ok = true;
-    while (ok && next_seg(p, t, t_end, cta, s)) {
-      if (wg < s.nm) {
-        float m = -INFINITY, l = 0.f;
-        for (int j = s.j0; j < s.j1; ++j) {
-          if (!(ok = warp_wait(B.s_full + wg, s_ph, abort_flag, p.wait_limit, p.status))) break;
-          s_ph ^= 1;
-          tc_fence_after();
-          uint32_t r[4][32];
-#pragma unroll
-          for (int c = 0; c < 4; ++c) tmem_ld32(t_S + c * 32, r[c]);
-          tmem_ld_wait();
-          const int kvalid = p.doc_len - j * kBN;  // keys of this tile inside the document
-          if (kvalid < kBN) {
-#pragma unroll
-            for (int c = 0; c < 4; ++c)
-#pragma unroll
-              for (int e = 0; e < 32; ++e)
-                if (c * 32 + e >= kvalid) r[c][e] = __float_as_uint(-INFINITY);
-          }
-          // row maximum: 8 independent chains of 3-input max
-          float mc[8];
-#pragma unroll
-          for (int k = 0; k < 8; ++k) mc[k] = -INFINITY;
-#pragma unroll
-          for (int i = 0; i < 128; i += 2)
-            mc[(i >> 1) & 7] = fmax3(mc[(i >> 1) & 7], __uint_as_float(r[i >> 5][i & 31]),
-                                     __uint_as_float(r[i >> 5][(i & 31) + 1]));
-          const float mx = fmax3(fmax3(mc[0], mc[1], mc[2]), fmax3(mc[3], mc[4], mc[5]),
-                                 fmaxf(mc[6], mc[7]));
-          const float m_new = fmaxf(m, mx * p.sl2);
-          // Lazy rescale: keep a stale maximum unless the new one exceeds it
-          // by more than 2^8 (probabilities then stay below 256).
-          const bool need = m_new > m + 8.f;
-          const float m_old = m;
-          if (need) {
-            l *= ex2_mufu(m - m_new);
-            m = m_new;
-          }
-          // P = 2^(S * scale*log2e - m) as bf16 pairs, written over S's first
-          // 64 columns chunk by chunk; row sum in 4 packed partial sums.
-          const float2 sl2v = make_float2(p.sl2, p.sl2), negm = make_float2(-m, -m);
-          float2 rs[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint32_t pk[16];
-#pragma unroll
-            for (int e = 0; e < 32; e += 2) {
-              const int pr_i = c * 16 + (e >> 1);
-              const float2 a = ffma2(make_float2(__uint_as_float(r[c][e]), __uint_as_float(r[c][e + 1])),
-                                     sl2v, negm);
-              float2 pv;
-              if (use_poly(pr_i)) {
-                pv = ex2_poly2(a);
-              } else {
-                pv.x = ex2_mufu(a.x);
-                pv.y = ex2_mufu(a.y);
-              }
-              rs[pr_i & 1] = fadd2(rs[pr_i & 1], pv);
-              pk[e >> 1] = f2_to_bf2(pv.x, pv.y);
-            }
-            tmem_st16(t_S + c * 16, pk);
-          }
-          l += (rs[0].x + rs[0].y) + (rs[1].x + rs[1].y);
-          // O rescale for rows whose maximum moved (rare; S is dead by now).
-          // O is stable here: O += P V of the previous tile has completed
-          // (committed before this tile's S) and this tile's is not issued
-          // before p_full.
-          if (j > s.j0 && __any_sync(0xffffffffu, need)) {
-            const float f = need ? ex2_mufu(m_old - m) : 1.f;
-#pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
-              uint32_t o[32];
-              tmem_ld32(t_O + c * 32, o);
-              tmem_ld_wait();
-#pragma unroll
-              for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
-              tmem_st32(t_O + c * 32, o);
-            }
-          }
-          tmem_st_wait();
-          tc_fence_before();
-          mbar_arrive(B.p_full + wg);
-        }
-        if (!ok) break;
-        // Epilogue: the segment's last O += P V has completed.
-        if (!(ok = warp_wait(B.o_done + wg, od_ph, abort_flag, p.wait_limit, p.status))) break;
-        od_ph ^= 1;
-        tc_fence_after();
-        const int row = s.g * kGroupRows + wg * 128 + rt;
-        const bool valid = row < p.rows;
-        const int64_t slot = (int64_t)s.u * p.plan.max_chunks + s.chunk;
-        const int64_t prow = slot * kGroupRows + wg * 128 + rt;
-        float4* dst = reinterpret_cast<float4*>(p.doc_o + prow * D);
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t o[32];
-          tmem_ld32(t_O + c * 32, o);
-          tmem_ld_wait();
-          if (valid) {
-#pragma unroll
-            for (int e = 0; e < 32; e += 4)
-              dst[(c * 32 + e) / 4] = make_float4(__uint_as_float(o[e]), __uint_as_float(o[e + 1]),
-                                                  __uint_as_float(o[e + 2]), __uint_as_float(o[e + 3]));
+    // Publish v for the partner half and return the partner's value of the
+    // same exchange (bounded spin; gives up on the abort flag or the limit).
+    auto swap_half = [&](float v, float& other) -> bool {
+      ++seq;
+      tc_fence_before();
+      volatile unsigned long long* mine = &xch[seq & 1][hf][rt];
+      volatile unsigned long long* theirs = &xch[seq & 1][hf ^ 1][rt];
+      *mine = ((unsigned long long)seq << 32) | __float_as_uint(v);
+      const long long t0 = clock64();
+      while (true) {
+        const unsigned long long x = *theirs;
+        const bool got = (uint32_t)(x >> 32) == seq;
+        if (got) other = __uint_as_float((uint32_t)x);
+        if (__all_sync(0xffffffffu, got)) break;
+        int stop = 0;
+        if (lane == 0) {
+          if (*abort_flag) {
+            stop = 1;
+          } else if (clock64() - t0 > p.wait_limit) {
+            *abort_flag = 1;
+            set_status(p.status, PP_DEV_TIMEOUT);
+            stop = 1;
           }
         }
-        if (valid) reinterpret_cast<float2*>(p.doc_ml)[prow] = make_float2(m, l);
-        tc_fence_before();
-        mbar_arrive(B.o_free + wg);
+        if (__shfl_sync(0xffffffffu, stop, 0)) return false;
       }
+      tc_fence_after();
+      return true;
+    };
+    while (ok && next_seg(p, t, t_end, slot, mt, s)) {
+      if (!s.active) continue;
+      float m = -INFINITY, l = 0.f;   // l: this half's share of the row sum
+      for (int j = s.j0; j < s.j1; ++j, ++g) {
+        const int b = (j - s.j0) & 1;
+        const uint32_t t_S = t_lane + C::T_S + (uint32_t)(b * kBN);
+        if (!(ok = warp_wait(B.s_full + b, (s_ph >> b) & 1, abort_flag, p.wait_limit, p.status)))
+          break;
+        s_ph ^= 1u << b;
+        tc_fence_after();
+        uint32_t r[2][32];
+#pragma unroll
+        for (int c = 0; c < 2; ++c) tmem_ld32(t_S + hf * HB + c * 32, r[c]);
+        tmem_ld_wait();
+        const int kvalid = p.doc_len - j * kBN - hf * HB;  // keys of this half inside the document
+        if (kvalid < HB) {
+#pragma unroll
+          for (int c = 0; c < 2; ++c)
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+              if (c * 32 + e >= kvalid) r[c][e] = __float_as_uint(-INFINITY);
+        }
+        // partial row maximum: 8 independent chains of 3-input max
+        float mc[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mc[k] = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < HB; i += 2)
+          mc[(i >> 1) & 7] = fmax3(mc[(i >> 1) & 7], __uint_as_float(r[i >> 5][i & 31]),
+                                   __uint_as_float(r[i >> 5][(i & 31) + 1]));
+        float mx = fmax3(fmax3(mc[0], mc[1], mc[2]), fmax3(mc[3], mc[4], mc[5]), fmaxf(mc[6], mc[7]));
+        // The swap also orders both halves' reads of S before either half's
+        // P overwrites columns the other half read.
+        float mo;
+        if (!(ok = swap_half(mx, mo))) break;
+        mx = fmaxf(mx, mo);
+        const float m_new = fmaxf(m, mx * p.sl2);
+        // Lazy rescale: keep a stale maximum unless the new one exceeds it
+        // by more than 2^8 (probabilities then stay below 256).  Both halves
+        // see the same maximum and take the same decision.
+        const bool need = m_new > m + 8.f;
+        const float m_old = m;
+        if (need) {
+          l *= ex2_mufu(m - m_new);
+          m = m_new;
+        }
+        // P = 2^(S * scale*log2e - m) as bf16 pairs, written over the S
+        // buffer's first 64 columns (this half's 32 of them).
+        const float2 sl2v = make_float2(p.sl2, p.sl2), negm = make_float2(-m, -m);
+        float2 rs[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const int pr_i = c * 16 + (e >> 1);
+            const float2 a = ffma2(make_float2(__uint_as_float(r[c][e]), __uint_as_float(r[c][e + 1])),
+                                   sl2v, negm);
+            float2 pv;
+            if (use_poly(pr_i)) {
+              pv = ex2_poly2(a);
+            } else {
+              pv.x = ex2_mufu(a.x);
+              pv.y = ex2_mufu(a.y);
+            }
+            rs[pr_i & 1] = fadd2(rs[pr_i & 1], pv);
+            pk[e >> 1] = f2_to_bf2(pv.x, pv.y);
+          }
+          tmem_st16(t_S + hf * (HB / 2) + c * 16, pk);
+        }
+        l += (rs[0].x + rs[0].y) + (rs[1].x + rs[1].y);
+        // O rescale for rows whose maximum moved (rare), this half's O
+        // columns.  The previous tile's O += P V may still run: wait for it
+        // (pv_done completes once per product, so its phase g - 1 is that
+        // one); this tile's is not issued before p_full.
+        if (j > s.j0 && __any_sync(0xffffffffu, need)) {
+          if (!(ok = warp_wait(B.pv_done, (g - 1) & 1, abort_flag, p.wait_limit, p.status))) break;
+          tc_fence_after();
+          const float f = need ? ex2_mufu(m_old - m) : 1.f;
+#pragma unroll
+          for (int c = 0; c < OC; ++c) {
+            uint32_t o[32];
+            tmem_ld32(t_O + c * 32, o);
+            tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
+            tmem_st32(t_O + c * 32, o);
+          }
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(B.p_full + b);
+      }
+      if (!ok) break;
+      // Epilogue: the segment's last O += P V has completed.
+      if (!(ok = warp_wait(B.o_done, od_ph, abort_flag, p.wait_limit, p.status))) break;
+      od_ph ^= 1;
+      tc_fence_after();
+      const int row = s.g * kGroupRows + mt * 128 + rt;
+      const bool valid = row < p.rows;
+      const int64_t pslot = (int64_t)s.u * p.plan.max_chunks + s.chunk;
+      const int64_t prow = pslot * kGroupRows + mt * 128 + rt;
+      float4* dst = reinterpret_cast<float4*>(p.doc_o + prow * D + hf * (D / 2));
+#pragma unroll
+      for (int c = 0; c < OC; ++c) {
+        uint32_t o[32];
+        tmem_ld32(t_O + c * 32, o);
+        tmem_ld_wait();
+        if (valid) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 4)
+            dst[(c * 32 + e) / 4] = make_float4(__uint_as_float(o[e]), __uint_as_float(o[e + 1]),
+                                                __uint_as_float(o[e + 2]), __uint_as_float(o[e + 3]));
+        }
+      }
+      float lo;
+      if (!(ok = swap_half(l, lo))) break;
+      if (valid && hf == 0) reinterpret_cast<float2*>(p.doc_ml)[prow] = make_float2(m, l + lo);
+      tc_fence_before();
+      mbar_arrive(B.o_free);
     }
   }
 
@@ -611,6 +655,7 @@ cudaError_t launch_impl(const pp_kv_layer& L, int doc_len, const uint16_t* q, in
   prm.rows = rows;
   prm.H = L.H;
   prm.G = (rows + kGroupRows - 1) / kGroupRows;
+  prm.pair = doc_pair_ctas(rows);
   prm.doc_len = doc_len;
   prm.plan = plan;
   prm.sl2 = scale * kLog2e;
@@ -619,7 +664,7 @@ cudaError_t launch_impl(const pp_kv_layer& L, int doc_len, const uint16_t* q, in
   prm.status = L.status;
   prm.wait_limit = wait_limit;
   prm.inject_timeout = inject;
-  doc_pass_tc<D><<<plan.C, 384, C::SMEM, st>>>(mQ, mK, mV, prm);
+  doc_pass_tc<D><<<plan.C * prm.pair, kThreads, C::SMEM, st>>>(mQ, mK, mV, prm);
   return cudaGetLastError();
 }
 

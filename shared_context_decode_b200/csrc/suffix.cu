@@ -209,10 +209,36 @@ __global__ void __launch_bounds__(SufCfg<D>::WARPS * 32) suffix_merge(const SufP
     for (int i = 0; i < C::NS - 1; ++i)
       if (issue_next(issued % C::NS)) ++issued;
 
+    // The query row and first-chunk tags of item k + 1 are loaded while item
+    // k runs, so no item starts on a global-memory round trip.
+    uint4 qn[C::G];
+    int sid0 = -1, pos0 = 0;
+    auto prefetch_item = [&](int k) {
+      const int64_t item = r0 + k;
+      const int h = (int)(item / p.rows), r = (int)(item - (int64_t)h * p.rows);
+      const uint4* qp4 = reinterpret_cast<const uint4*>(p.q + ((int64_t)r * p.H + h) * D);
+#pragma unroll
+      for (int c = 0; c < C::G; ++c) qn[c] = __ldg(qp4 + g + 8 * c);
+      const ItemRec rec = tbl[k];
+      sid0 = -1;
+      pos0 = 0;
+      if (my_key < rec.n) {
+        sid0 = __ldg(p.sid + (size_t)(rec.s - 1) * p.S_cap + my_key);
+        pos0 = __ldg(p.pos + (size_t)(rec.s - 1) * p.S_cap + my_key);
+      }
+    };
+    if (cnt > 0) prefetch_item(0);
+
     for (int k = 0; k < cnt; ++k) {
       const int64_t item = r0 + k;
       const int h = (int)(item / p.rows), r = (int)(item - (int64_t)h * p.rows);
       const ItemRec rec = tbl[k];
+      uint4 qr[C::G];
+#pragma unroll
+      for (int c = 0; c < C::G; ++c) qr[c] = qn[c];
+      // this lane's key tags, loaded one chunk ahead of their use
+      int nsid = sid0, npos = pos0;
+      if (k + 1 < cnt) prefetch_item(k + 1);
       const bool valid = rec.s != 0;
       // document partials of this (row, head), fetched now so their latency
       // hides behind the segment's chunks
@@ -246,10 +272,9 @@ __global__ void __launch_bounds__(SufCfg<D>::WARPS * 32) suffix_merge(const SufP
       // this lane's query dims (groups g, g + 8, ...), scaled by scale * log2(e)
       float2 q2[C::G * 4];
       {
-        const uint4* qp4 = reinterpret_cast<const uint4*>(p.q + ((int64_t)r * p.H + h) * D);
 #pragma unroll
         for (int c = 0; c < C::G; ++c) {
-          const uint4 w = qp4[g + 8 * c];
+          const uint4 w = qr[c];
           const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
@@ -264,12 +289,6 @@ __global__ void __launch_bounds__(SufCfg<D>::WARPS * 32) suffix_merge(const SufP
       const int16_t* sb = p.sid + (size_t)(valid ? rec.s - 1 : 0) * p.S_cap;
       const int32_t* pb = p.pos + (size_t)(valid ? rec.s - 1 : 0) * p.S_cap;
 
-      // this lane's key tags, loaded one chunk ahead of their use
-      int nsid = -1, npos = 0;
-      if (my_key < rec.n) {
-        nsid = __ldg(sb + my_key);
-        npos = __ldg(pb + my_key);
-      }
       for (int t0 = 0; t0 < rec.n; t0 += C::CK) {
         if (issue_next(issued % C::NS)) ++issued;
         const int t = t0 + my_key;
