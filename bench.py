@@ -15,6 +15,16 @@ the 126 MB L2, so no flush is needed between steps.
 Output: one JSON line on rank 0 (see the keys in main()).  Multi-GPU
 (torchrun): every rank runs an independent replica (weak scaling, no data
 collective); time is the max over ranks.
+
+Secondary measurements (--mode, one GPU, one JSON line each):
+  prefill   question prefill of the prefill_doc12k_p256 workload: per layer,
+            append the R question rows, then pp_prefill_attn; rows/s and the
+            document part's TFLOP/s
+  ablation  the decode step with the per-stream document pass (every stream
+            reads the whole document) instead of the shared one
+  sweep     answer generation over doc x streams: 32 decode steps x 32
+            layers per combination, streams stopping after geometric lengths
+            (inactive rows keep their place in the fixed-shape graph)
 """
 from __future__ import annotations
 
@@ -169,6 +179,7 @@ class DecodeStep:
             del L
         torch.cuda.synchronize()
         self.len0 = self.len_all.clone()
+        self.opts = None   # per-layer pp_options of the captured step (None = default)
         self.ws = pp.workspace(pp.decode_workspace_bytes(W.P, W.H, W.d, W.N), device)
         self.graph = None
 
@@ -176,6 +187,7 @@ class DecodeStep:
         """One decode step, launched eagerly (also the body that is captured);
         opts: per-layer pp_options or None."""
         pp = self.pp
+        opts = opts if opts is not None else self.opts
         self.len_all.copy_(self.len0)
         for l in range(self.layers):
             x = self.inp[l]
@@ -210,6 +222,230 @@ class DecodeStep:
                 raise RuntimeError(f"device status {st:#x}")
 
 
+class PrefillStep:
+    """Question prefill of all layers as one CUDA graph: per layer, append the
+    R question rows to their stream segments (emptied at the start of every
+    step), then pp_prefill_attn (document pass with M = 128-row tiles of all
+    R rows, the causal question part, merge)."""
+
+    def __init__(self, name: str, layers: int, device, seed: int = 0):
+        from shared_context_decode_b200 import ppattn as pp
+        from shared_context_decode_b200 import workloads as wl
+        self.pp = pp
+        self.W = W = wl.make_prefill(name, seed=seed, device=device)
+        self.layers = layers
+        self.device = device
+        S_cap = int(math.ceil(int(W.q_len.max()) / 16) * 16)
+        self.len_all = torch.zeros((layers, W.P), dtype=torch.int32, device=device)
+        self.cache, self.inp = [], []
+        for l in range(layers):
+            L = W.layer(l)
+            kv = pp.KVLayer(W.H, W.d, W.N, W.P, S_cap, device, len_buf=self.len_all[l])
+            pp.kv_append(kv, L.doc_k, L.doc_v, torch.zeros(W.N, dtype=torch.int16, device=device),
+                         torch.arange(W.N, dtype=torch.int32, device=device))
+            self.cache.append(kv)
+            self.inp.append(dict(k=L.qk, v=L.qv, q=L.q, sid=L.sid, pos=L.pos,
+                                 o=torch.empty_like(L.q)))
+            del L
+        torch.cuda.synchronize()
+        self.ws = pp.workspace(pp.prefill_workspace_bytes(W.R, W.H, W.d, W.N), device)
+        self.graph = None
+
+    def run_eager(self):
+        pp = self.pp
+        self.len_all.zero_()
+        for l in range(self.layers):
+            x = self.inp[l]
+            pp.kv_append(self.cache[l], x["k"], x["v"], x["sid"], x["pos"])
+            pp.prefill_attn(self.cache[l], self.W.N, x["q"], x["sid"], x["pos"], self.W.scale,
+                            o=x["o"], ws=self.ws)
+
+    capture = DecodeStep.capture
+    replay = DecodeStep.replay
+    check_status = DecodeStep.check_status
+
+    def kernels_per_step(self) -> int:
+        return self.layers * 4
+
+
+def timed_replays(step, steps: int, warmup: int, world: int, local: int):
+    for _ in range(warmup):
+        step.replay()
+    torch.cuda.synchronize()
+    barrier(world)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clocks:
+        torch.cuda.synchronize()
+        clocks.mark("start")
+        t0.record()
+        for _ in range(steps):
+            step.replay()
+        t1.record()
+        torch.cuda.synchronize()
+        clocks.mark("end")
+    barrier(world)
+    return t0.elapsed_time(t1) / steps, clocks.summary()
+
+
+def mode_prefill(args, world, rank, local, dev):
+    name = "prefill_doc12k_p256"
+    from shared_context_decode_b200 import workloads as wl
+    nl = args.layers or wl.CONFIGS[name]["layers"]
+    step = PrefillStep(name, nl, dev)
+    step.capture()
+    W = step.W
+    ms, clocks = timed_replays(step, args.steps, args.warmup, world, local)
+    step.check_status()
+    value, ms = aggregate(W.R, ms, world, dev)
+    flops = 4.0 * W.R * W.N * W.d * W.H * nl
+    tfs = flops / (ms / 1e3) / 1e12 * world
+    peaks = load_peaks()
+    line = {"mode": "prefill", "metric": "prefill rows/s", "value": value, "unit": "rows/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": name, "layers": nl, "H": W.H, "d": W.d, "doc_tokens": W.N,
+                       "streams": W.P, "rows": W.R,
+                       "l2": "per-layer document KV and question rows exceed L2"},
+            "doc_tflops": tfs, "doc_frac_of_sustained_bf16": tfs / world / peaks["bf16_sustained"],
+            "gpu_launches": step.kernels_per_step() * args.steps, "clocks": clocks}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    del step.graph
+
+
+def mode_ablation(args, world, rank, local, dev):
+    from shared_context_decode_b200 import workloads as wl
+    nl = args.layers or 4
+    step = DecodeStep(args.workload, nl, dev)
+    pp = step.pp
+    step.opts = [pp.Options(ablation_doc_per_stream=1) for _ in range(nl)]
+    step.capture()
+    W = step.W
+    ms, clocks = timed_replays(step, args.steps, args.warmup, world, local)
+    step.check_status()
+    value, ms = aggregate(W.P, ms, world, dev)
+    shared_b, _ = doc_pass_algorithmic(W)
+    line = {"mode": "ablation", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": args.workload, "layers": nl, "H": W.H, "d": W.d,
+                       "doc_tokens": W.N, "streams": W.P, "ablation": "doc_per_stream"},
+            "doc_bytes_per_layer_shared": shared_b, "doc_bytes_per_layer_ablation": shared_b * W.P,
+            "gpu_launches": step.kernels_per_step() * args.steps, "clocks": clocks}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    del step.graph
+
+
+def sweep_combo(N: int, P: int, layers: int, dev, warm: bool = True):
+    """One doc x streams combination of the answer-generation sweep: returns
+    (active stream-tokens, device ms) over its decode steps.  The graph holds
+    all P rows; a stream past its stop length keeps its row with stream id -1
+    (no append, no suffix work, zero output)."""
+    from shared_context_decode_b200 import ppattn as pp
+    from shared_context_decode_b200 import workloads as wl
+    cfg = wl.sweep_config(N, P)
+    name = f"sweep_N{N}_P{P}"
+    W = wl.make_decode(None, layers=layers, H=cfg["H"], d=cfg["d"], N=N, P=P, q=cfg["q"],
+                       a=cfg["a"], device=dev)
+    stops = wl.stop_lengths(P, name)
+    steps = cfg["steps"]
+    S_cap = int(math.ceil((int(W.q_len.max()) + steps + 1) / 16) * 16)
+    len_all = torch.zeros((layers, P), dtype=torch.int32, device=dev)
+    cache, inp = [], []
+    for l in range(layers):
+        L = W.layer(l)
+        kv = pp.KVLayer(W.H, W.d, N, P, S_cap, dev, len_buf=len_all[l])
+        pp.kv_append(kv, L.doc_k, L.doc_v, torch.zeros(N, dtype=torch.int16, device=dev),
+                     torch.arange(N, dtype=torch.int32, device=dev))
+        pp.kv_append(kv, L.suf_k, L.suf_v, L.suf_sid, L.suf_pos)
+        cache.append(kv)
+        inp.append(dict(k=L.new_k, v=L.new_v, q=L.q, o=torch.empty_like(L.q)))
+        del L
+    torch.cuda.synchronize()
+    len0 = len_all.clone()
+    q_sid = torch.empty(P, dtype=torch.int16, device=dev)
+    q_pos = torch.empty(P, dtype=torch.int32, device=dev)
+    ws = pp.workspace(pp.decode_workspace_bytes(P, W.H, W.d, N), dev)
+    base_pos = (N + W.q_len).astype(np.int32)
+    sids = np.arange(1, P + 1, dtype=np.int16)
+    host = [(torch.from_numpy(np.where(t < stops, sids, -1).astype(np.int16)).pin_memory(),
+             torch.from_numpy(base_pos + t).pin_memory(), int((t < stops).sum()))
+            for t in range(steps)]
+
+    def body():
+        for l in range(layers):
+            x = inp[l]
+            pp.kv_append(cache[l], x["k"], x["v"], q_sid, q_pos)
+            pp.decode_attn(cache[l], N, x["q"], q_sid, q_pos, W.scale, o=x["o"], ws=ws)
+
+    q_sid.copy_(host[0][0])
+    q_pos.copy_(host[0][1])
+    body()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream(dev)
+    s.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            body()
+    torch.cuda.current_stream(dev).wait_stream(s)
+    torch.cuda.synchronize()
+    tokens, ms = 0, 0.0
+    for rep in range(2 if warm else 1):
+        len_all.copy_(len0)
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(steps)]
+        for t in range(steps):
+            q_sid.copy_(host[t][0], non_blocking=True)
+            q_pos.copy_(host[t][1], non_blocking=True)
+            ev[t][0].record()
+            g.replay()
+            ev[t][1].record()
+        torch.cuda.synchronize()
+        tokens = sum(h[2] for h in host)
+        ms = sum(a.elapsed_time(b) for a, b in ev)
+    for kv in cache:
+        st = pp.device_status(kv)
+        if st:
+            raise RuntimeError(f"device status {st:#x} in sweep N={N} P={P}")
+    # every stream appended exactly min(stop, steps) tokens
+    want = len0.cpu() + torch.from_numpy(np.minimum(stops, steps).astype(np.int32))
+    if not torch.equal(len_all.cpu(), want):
+        raise RuntimeError(f"segment lengths after the sweep differ (N={N} P={P})")
+    del g
+    return tokens, ms, float(np.mean(stops))
+
+
+def mode_sweep(args, world, rank, local, dev):
+    from shared_context_decode_b200 import workloads as wl
+    nl = args.layers or 32
+    rows, tot_tok, tot_ms = [], 0, 0.0
+    with ClockSampler(local) as clocks:
+        clocks.mark("start")
+        for N in wl.SWEEP_DOCS:
+            for P in wl.SWEEP_STREAMS:
+                tok, ms, mean_stop = sweep_combo(N, P, nl, dev)
+                torch.cuda.empty_cache()
+                rows.append({"N": N, "P": P, "stream_tokens": tok, "ms": ms,
+                             "value": tok / (ms / 1e3), "mean_stop": mean_stop})
+                tot_tok += tok
+                tot_ms += ms
+        clocks.mark("end")
+    value, ms = aggregate(tot_tok, tot_ms, world, dev)
+    line = {"mode": "sweep", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": wl.SWEEP_STEPS, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "sweep", "layers": nl, "docs": list(wl.SWEEP_DOCS),
+                       "streams": list(wl.SWEEP_STREAMS),
+                       "stops": f"min({wl.SWEEP_STOP_CAP}, Geometric(1/{wl.SWEEP_STOP_MEAN}))"},
+            "combos": rows, "clocks": clocks.summary()}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def doc_pass_algorithmic(W):
     """Algorithmic bytes and FLOPs of one document-pass launch (one layer):
     every document K and V byte read once; S = Q K^T and O = P V over all
@@ -217,6 +453,38 @@ def doc_pass_algorithmic(W):
     bytes_ = 2 * W.N * W.H * W.d * 2
     flops = 4 * W.P * W.N * W.d * W.H
     return bytes_, flops
+
+
+DOC_PROFILE = os.path.join(ROOT, "profiles", "doc_pass_tc_doc16k_p256.md")
+DOC_SOURCES = ("doc_tc.cu", "common.cuh")
+
+
+def kernel_source_hash(files=DOC_SOURCES) -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, "shared_context_decode_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def profile_traffic(path: str = DOC_PROFILE, files=DOC_SOURCES):
+    """DRAM bytes (read + write) per launch from a committed ncu summary, or
+    None when the summary is absent or the kernel's sources changed since
+    the capture (the summary records their sha256)."""
+    if not os.path.exists(path):
+        return None
+    fields = {}
+    for line in open(path).read().splitlines():
+        if ":" in line and line.startswith("- "):
+            k, v = line[2:].split(":", 1)
+            fields[k.strip()] = v.strip().strip("`")
+    try:
+        if fields.get("sources sha256") != kernel_source_hash(files):
+            return None
+        return float(fields["dram bytes per launch (read + write)"])
+    except (KeyError, ValueError):
+        return None
 
 
 def load_peaks():
@@ -331,6 +599,8 @@ def main():
                     help="CPU-baseline sample budget (0 = skip)")
     ap.add_argument("--ref-seconds", type=float, default=10.0)
     ap.add_argument("--roofline-reps", type=int, default=3)
+    ap.add_argument("--mode", default="decode", choices=["decode", "prefill", "ablation", "sweep"],
+                    help="decode: the headline step (default); others: secondary measurements")
     args = ap.parse_args()
     world, rank, local = dist_env()
     if world > 1:
@@ -347,6 +617,13 @@ def main():
     assert args.warmup >= 3, "at least 3 warm-up steps"
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
+    if args.mode != "decode":
+        {"prefill": mode_prefill, "ablation": mode_ablation, "sweep": mode_sweep}[args.mode](
+            args, world, rank, local, dev)
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return
     from shared_context_decode_b200 import workloads as wl
     nl = args.layers or wl.CONFIGS[args.workload]["layers"]
     step = DecodeStep(args.workload, nl, dev)
@@ -414,7 +691,7 @@ def main():
     else:
         roof = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm"], "unit": "GB/s",
                 "frac": gbs / peaks["hbm"]}
-    roof.update({"traffic": None, "kernel": "pp::doc_pass_tc<128>",
+    roof.update({"traffic": profile_traffic(), "kernel": "pp::doc_pass_tc<128>",
                  "peak_source": peaks["source"] + (" sustained bf16" if roof["bound"] == "tensor"
                                                    else " copy"),
                  "doc_us": durs["doc"] * 1e3, "suffix_merge_us": durs["suffix"] * 1e3,
