@@ -1,0 +1,88 @@
+"""The bench's multi-rank plumbing on CPU (gloo, world size 2): every rank runs
+an independent replica; the whole-job value is the units of all ranks over the
+slowest rank's time, and only rank 0 prints the reference arm."""
+import os
+import socket
+import sys
+
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def rank_main(rank, world, port, out):
+    import datetime
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    import bench
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        dev = torch.device("cpu")
+        ms_rank = [4.0, 5.0][rank]          # rank 1 is the slower replica
+        units_rank = [256.0, 256.0][rank]
+        value, ms = bench.aggregate(units_rank, ms_rank, world, dev)
+        mx = bench.reduce_max(float(rank) + 0.5, world, dev)
+        sm = bench.reduce_sum(float(rank) + 1.0, world, dev)
+        bench.barrier(world)
+        out[rank] = (value, ms, mx, sm)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_aggregate_over_two_gloo_ranks():
+    ctx = mp.get_context("spawn")
+    out = ctx.Manager().dict()
+    mp.start_processes(rank_main, args=(2, free_port(), out), nprocs=2, join=True,
+                       start_method="spawn")
+    assert set(out.keys()) == {0, 1}
+    for rank in (0, 1):
+        value, ms, mx, sm = out[rank]
+        assert ms == 5.0                      # the slowest rank's time
+        assert value == pytest.approx(512.0 / 5e-3)   # all ranks' units / that time
+        assert mx == 1.5 and sm == 3.0
+
+
+def test_reference_arm_runs_on_rank_zero_only(capsys):
+    sys.path.insert(0, ROOT)
+    import bench
+
+    class Args:
+        workload = "tiny"
+        steps = 1
+        warmup = 0
+        ref_seconds = 0.01
+
+    bench.reference_arm(Args, world=2, rank=1)
+    assert capsys.readouterr().out == ""
+
+
+def test_reference_arm_line_on_rank_zero(capsys):
+    """--impl reference: the oracle timed on the host, one JSON line with the
+    contract's keys (a bounded sample of the tiny workload)."""
+    import json
+    sys.path.insert(0, ROOT)
+    import bench
+
+    class Args:
+        workload = "tiny"
+        steps = 2
+        warmup = 1
+        ref_seconds = 0.01
+
+    bench.reference_arm(Args, world=1, rank=0)
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["value"] > 0
+    assert line["e2e"] == {"value": line["value"], "unit": line["unit"],
+                           "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+    assert line["config"]["workload"] == "tiny"
