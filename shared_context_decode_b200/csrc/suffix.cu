@@ -35,7 +35,8 @@ namespace pp {
 
 template <int D>
 struct SufCfg {
-  static constexpr int CK = 16;              // keys per chunk
+  static constexpr int CK = 16;              // keys per chunk (8 or 16)
+  static constexpr int NPASS = CK / 4;       // score passes of 4 keys
   static constexpr int ROWB = D * 2;         // bytes of one key row
   static constexpr int HALF = CK * ROWB;     // K (or V) part of a stage
   static constexpr int STAGE = 2 * HALF;
@@ -123,8 +124,12 @@ __device__ __forceinline__ bool stage_wait(uint64_t* bar, uint32_t parity, volat
   }
 }
 
-// Lane holding the score of chunk key kk after the transpose-reduce.
-__device__ __forceinline__ int key_lane(int kk) { return (kk & 3) * 8 + (kk >> 2) * 2; }
+// Lane holding the score of chunk key kk after the transpose-reduce (of
+// NPASS passes of 4 keys).
+template <int NPASS>
+__device__ __forceinline__ int key_lane(int kk) {
+  return (kk & 3) * 8 + (kk >> 2) * (8 / NPASS);
+}
 
 template <int D>
 __global__ void __launch_bounds__(SufCfg<D>::WARPS * 32) suffix_merge(const SufParams p) {
@@ -137,7 +142,8 @@ __global__ void __launch_bounds__(SufCfg<D>::WARPS * 32) suffix_merge(const SufP
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane & 7, sub = lane >> 3;          // score: 16-byte group, key of a pass
   const int b2 = (lane >> 2) & 1, b1 = (lane >> 1) & 1;
-  const int my_key = 4 * (2 * b2 + b1) + sub;       // key whose score this lane ends with
+  // key whose score this lane ends with
+  const int my_key = C::NPASS == 4 ? 4 * (2 * b2 + b1) + sub : 4 * b2 + sub;
   uint8_t* ring = smem + warp * C::NS * C::STAGE;
   ItemRec* tbl = reinterpret_cast<ItemRec*>(smem + C::WARPS * C::NS * C::STAGE) + warp * C::TBL;
   uint64_t* full = bars[warp];
@@ -306,9 +312,9 @@ __global__ void __launch_bounds__(SufCfg<D>::WARPS * 32) suffix_merge(const SufP
         const uint8_t* sV = sK + C::HALF;
         // partial dots of keys 4 j + sub (pass j) over this lane's groups;
         // rows past the chunk's live keys hold stale bytes and are masked below
-        float v[4];
+        float v[C::NPASS];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
+        for (int j = 0; j < C::NPASS; ++j) {
           const uint8_t* rowp = sK + (4 * j + sub) * C::ROWB + g * 16;
           float2 d0 = make_float2(0.f, 0.f), d1 = make_float2(0.f, 0.f);
 #pragma unroll
@@ -334,25 +340,32 @@ __global__ void __launch_bounds__(SufCfg<D>::WARPS * 32) suffix_merge(const SufP
             vw[kk][0] = *reinterpret_cast<const uint32_t*>(sV + kk * C::ROWB + lane * 4);
           }
         }
-        // transpose-reduce over the 8 lanes of a key group: xor 4 splits the
-        // passes {0,1} | {2,3}, xor 2 splits the pair, xor 1 finishes the sum
-        float w0, w1;
-        {
-          const float r0s = __shfl_xor_sync(0xffffffffu, b2 ? v[0] : v[2], 4);
-          const float r1s = __shfl_xor_sync(0xffffffffu, b2 ? v[1] : v[3], 4);
-          w0 = (b2 ? v[2] : v[0]) + r0s;
-          w1 = (b2 ? v[3] : v[1]) + r1s;
+        // transpose-reduce over the 8 lanes of a key group.  Four passes:
+        // xor 4 splits the passes {0,1} | {2,3}, xor 2 splits the pair, xor 1
+        // finishes the sum.  Two passes: xor 4 splits them, xor 2 and xor 1
+        // finish the sum.
+        float dot;
+        if constexpr (C::NPASS == 4) {
+          const float r0s = __shfl_xor_sync(0xffffffffu, b2 ? v[0] : v[2 % C::NPASS], 4);
+          const float r1s = __shfl_xor_sync(0xffffffffu, b2 ? v[1] : v[3 % C::NPASS], 4);
+          const float w0 = (b2 ? v[2 % C::NPASS] : v[0]) + r0s;
+          const float w1 = (b2 ? v[3 % C::NPASS] : v[1]) + r1s;
+          dot = (b1 ? w1 : w0) + __shfl_xor_sync(0xffffffffu, b1 ? w0 : w1, 2);
+        } else {
+          dot = (b2 ? v[1] : v[0]) + __shfl_xor_sync(0xffffffffu, b2 ? v[0] : v[1], 4);
+          dot += __shfl_xor_sync(0xffffffffu, dot, 2);
         }
-        float dot = (b1 ? w1 : w0) + __shfl_xor_sync(0xffffffffu, b1 ? w0 : w1, 2);
         dot += __shfl_xor_sync(0xffffffffu, dot, 1);
         const float x = slot_visible(rec.s, rec.qp, tsid, tpos, t, rec.n) ? dot : -INFINITY;
+        // chunk maximum over the lanes holding distinct keys
         float cm = fmaxf(m, x);
 #pragma unroll
-        for (int o = 2; o < 32; o <<= 1) cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, o));
+        for (int o = 8 / C::NPASS; o < 32; o <<= 1) cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, o));
         if (cm != -INFINITY) {  // warp-uniform
           const float corr = exp2f(m - cm);  // m = -inf gives 0
           const float pr = exp2f(x - cm);    // masked keys give 0
-          lp = lp * corr + ((lane & 1) ? 0.f : pr);
+          // each key's probability sits on 8 / NPASS lanes: count it once
+          lp = lp * corr + ((lane & (8 / C::NPASS - 1)) ? 0.f : pr);
           const uint32_t live = __ballot_sync(0xffffffffu, pr > 0.f);
           float2 a2[C::E / 2];
 #pragma unroll
@@ -361,8 +374,8 @@ __global__ void __launch_bounds__(SufCfg<D>::WARPS * 32) suffix_merge(const SufP
           // a segment's end hold stale data)
 #pragma unroll
           for (int kk = 0; kk < C::CK; ++kk) {
-            const float pk = __shfl_sync(0xffffffffu, pr, key_lane(kk));
-            const bool on = (live >> key_lane(kk)) & 1u;
+            const float pk = __shfl_sync(0xffffffffu, pr, key_lane<C::NPASS>(kk));
+            const bool on = (live >> key_lane<C::NPASS>(kk)) & 1u;
             const float2 pk2 = make_float2(pk, pk);
 #pragma unroll
             for (int e = 0; e < C::E / 2; ++e) a2[e] = ffma2(pk2, bf2_to_f2(on ? vw[kk][e] : 0u), a2[e]);
