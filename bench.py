@@ -26,6 +26,8 @@ Secondary measurements (--mode, one GPU, one JSON line each):
             document part's TFLOP/s
   ablation  the decode step with the per-stream document pass (every stream
             reads the whole document) instead of the shared one
+  docprefill  causal attention of a 16384-token document over its own
+            tokens (pp_doc_prefill_attn), 32 heads, d = 128; tokens/s and TFLOP/s
   sweep     answer generation over doc x streams: 32 decode steps x 32
             layers per combination, streams stopping after geometric lengths
             (inactive rows keep their place in the fixed-shape graph)
@@ -385,6 +387,56 @@ def mode_ablation(args, world, rank, local, dev):
     del step.graph
 
 
+def mode_docprefill(args, world, rank, local, dev):
+    """Document prefill: per layer, causal attention of the document's own
+    tokens with the document K/V already cached (written once, outside the
+    timed region, as the append of the document would)."""
+    from shared_context_decode_b200 import ppattn as pp
+    from shared_context_decode_b200 import workloads as wl
+    N, H, d = 16384, 32, 128
+    nl = args.layers or 8
+    layers, inp = [], []
+    for l in range(nl):
+        k = wl.randn_bf16((N, H, d), wl.seed_of("docprefill", l, "k"), dev)
+        v = wl.randn_bf16((N, H, d), wl.seed_of("docprefill", l, "v"), dev)
+        kv = pp.KVLayer(H, d, N, 1, 16, dev)
+        pp.kv_append(kv, k, v, torch.zeros(N, dtype=torch.int16, device=dev),
+                     torch.arange(N, dtype=torch.int32, device=dev))
+        del k, v
+        q = wl.randn_bf16((N, H, d), wl.seed_of("docprefill", l, "q"), dev)
+        layers.append(kv)
+        inp.append((q, torch.empty_like(q)))
+    ws = pp.workspace(pp.doc_prefill_workspace_bytes(H, d, N), dev)
+    scale = 1.0 / math.sqrt(d)
+
+    class Step:
+        def run_eager(self):
+            for l in range(nl):
+                pp.doc_prefill_attn(layers[l], N, inp[l][0], scale, o=inp[l][1], ws=ws)
+
+    step = Step()
+    step.device, step.cache, step.pp = dev, layers, pp
+    DecodeStep.capture(step)
+    step.replay = lambda: step.graph.replay()
+    ms, clocks = timed_replays(step, args.steps, args.warmup, world, local)
+    DecodeStep.check_status(step)
+    value, ms = aggregate(N * nl, ms, world, dev)
+    flops = 4.0 * d * H * (N * (N + 1) / 2) * nl   # the causal half of S = QK^T and O = PV
+    tfs = flops / (ms / 1e3) / 1e12 * world
+    peaks = load_peaks()
+    line = {"mode": "docprefill", "metric": "document-prefill tokens/s", "value": value,
+            "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "document prefill", "layers": nl, "H": H, "d": d,
+                       "doc_tokens": N},
+            "tflops": tfs, "frac_of_sustained_bf16": tfs / world / peaks["bf16_sustained"],
+            "gpu_launches": 2 * nl * args.steps, "clocks": clocks}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    del step.graph
+
+
 def sweep_combo(N: int, P: int, layers: int, dev, warm: bool = True):
     """One doc x streams combination of the answer-generation sweep: returns
     (active stream-tokens, device ms) over its decode steps.  The graph holds
@@ -645,7 +697,8 @@ def main():
                     help="CPU-baseline sample budget (0 = skip)")
     ap.add_argument("--ref-seconds", type=float, default=10.0)
     ap.add_argument("--roofline-reps", type=int, default=3)
-    ap.add_argument("--mode", default="decode", choices=["decode", "prefill", "ablation", "sweep"],
+    ap.add_argument("--mode", default="decode",
+                    choices=["decode", "prefill", "ablation", "sweep", "docprefill"],
                     help="decode: the headline step (default); others: secondary measurements")
     args = ap.parse_args()
     world, rank, local = dist_env()
@@ -664,7 +717,8 @@ def main():
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     if args.mode != "decode":
-        {"prefill": mode_prefill, "ablation": mode_ablation, "sweep": mode_sweep}[args.mode](
+        {"prefill": mode_prefill, "ablation": mode_ablation, "sweep": mode_sweep,
+         "docprefill": mode_docprefill}[args.mode](
             args, world, rank, local, dev)
         if world > 1:
             import torch.distributed as dist

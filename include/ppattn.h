@@ -226,6 +226,31 @@ pp_status pp_prefill_attn(const pp_kv_layer *layer, int32_t doc_len, const uint1
                           uint16_t *o, float *lse, void *ws, size_t ws_bytes,
                           const pp_options *opt, void *stream);
 
+/* Workspace bytes pp_doc_prefill_attn needs for a document of doc_len tokens. */
+size_t pp_doc_prefill_workspace_bytes(int32_t H, int32_t d, int32_t doc_len,
+                                      const pp_options *opt);
+
+/*
+ * Document prefill: attention of the document's own tokens, done once for
+ * all streams ("Read Once, Answer Many" project page, section "How it
+ * works": the document is encoded once and shared; a document token, stream
+ * id 0, sees the document tokens at or before its own position, i.e.
+ * ordinary causal attention over the document).
+ *   q   bf16 [doc_len][H][d]  query of document token i at row i (position i)
+ *   o   bf16 [doc_len][H][d], lse fp32 [doc_len][H] or NULL
+ *   ws  caller-owned, 256-byte aligned, >= pp_doc_prefill_workspace_bytes
+ * The document's K/V rows 0 .. doc_len-1 must already be in the layer
+ * (pp_kv_append with stream id 0).  Runs on the same tensor-core document
+ * pass as decode, with row i masked to keys 0..i and the key tiles above a
+ * row group's diagonal skipped; the per-stream ablation option is refused
+ * (PP_ERR_UNSUPPORTED).  Other errors as for pp_decode_attn.  This call has
+ * no counterpart in the pages' measurements; their document prefill runs in
+ * the serving engine.
+ */
+pp_status pp_doc_prefill_attn(const pp_kv_layer *layer, int32_t doc_len, const uint16_t *q,
+                              float scale, uint16_t *o, float *lse, void *ws, size_t ws_bytes,
+                              const pp_options *opt, void *stream);
+
 /*
  * Test aid: evaluate the mask predicate the attention kernels use.
  *   count_out int32 [nq]: number of keys query i sees (document included).
@@ -246,6 +271,15 @@ pp_status pp_debug_visibility(const pp_kv_layer *layer, int32_t doc_len, const i
  */
 pp_status pp_debug_split_plan(int32_t rows, int32_t H, int32_t doc_len, int32_t ctas,
                               int64_t *h_out, int32_t h_out_len);
+
+/*
+ * Test aid (host only): the split pp_doc_prefill_attn uses for a document of
+ * doc_len tokens (rows = doc_len; unit (head, group g) holds only the key
+ * tiles 0 .. min(T, 2g+2)-1).  Same output layout as pp_debug_split_plan,
+ * with h_out[0] = T of a full unit.
+ */
+pp_status pp_debug_split_plan_causal(int32_t doc_len, int32_t H, int32_t ctas, int64_t *h_out,
+                                     int32_t h_out_len);
 
 /*
  * Test aid: the document pass's two base-2 exponentials on n device floats:

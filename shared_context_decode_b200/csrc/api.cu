@@ -50,12 +50,15 @@ pp_status check_layer(const pp_kv_layer* L) {
 
 pp_status from_cuda(cudaError_t e) { return e == cudaSuccess ? PP_OK : PP_ERR_CUDA; }
 
-// The document split: see pp::SplitPlan.  `ctas` = CTAs to spread it over.
-SplitPlan make_plan(int rows, int H, int doc_len, int ctas) {
+// The document split: see pp::SplitPlan.  `ctas` = slots to spread it over;
+// `causal`: a document prefill (rows = document tokens, triangular units).
+SplitPlan make_plan(int rows, int H, int doc_len, int ctas, bool causal = false) {
   SplitPlan p{};
   p.T = (doc_len + pp::kBN - 1) / pp::kBN;
-  p.units = ((rows + pp::kGroupRows - 1) / pp::kGroupRows) * H;
-  p.W = (int64_t)p.units * p.T;
+  p.G = (rows + pp::kGroupRows - 1) / pp::kGroupRows;
+  p.units = p.G * H;
+  p.causal = causal ? 1 : 0;
+  p.W = p.G > 0 && p.T > 0 ? (int64_t)H * pp::plan_head_tiles(p) : 0;
   if (p.W == 0 || ctas < 1) {
     p.C = 0;
     p.max_chunks = 0;
@@ -64,7 +67,9 @@ SplitPlan make_plan(int rows, int H, int doc_len, int ctas) {
   p.C = (int32_t)std::min<int64_t>(ctas, p.W);
   int mc = 1;
   for (int u = 0; u < p.units; ++u) {
-    const int n = pp::plan_cta_of(p, (int64_t)u * p.T + p.T - 1) - pp::plan_cta_of(p, (int64_t)u * p.T) + 1;
+    const int64_t ub = pp::plan_unit_begin(p, u);
+    const int n = pp::plan_cta_of(p, ub + pp::plan_unit_tiles(p, u % p.G) - 1) -
+                  pp::plan_cta_of(p, ub) + 1;
     mc = std::max(mc, n);
   }
   p.max_chunks = mc;
@@ -74,7 +79,8 @@ SplitPlan make_plan(int rows, int H, int doc_len, int ctas) {
 // The ablation reads the whole document per row: one chunk per unit.
 SplitPlan ablation_plan(int rows, int H, int doc_len) {
   SplitPlan p{};
-  p.units = ((rows + pp::kGroupRows - 1) / pp::kGroupRows) * H;
+  p.G = (rows + pp::kGroupRows - 1) / pp::kGroupRows;
+  p.units = p.G * H;
   p.T = doc_len > 0 ? 1 : 0;
   p.W = (int64_t)p.units * p.T;
   p.C = (int32_t)p.W;
@@ -82,12 +88,12 @@ SplitPlan ablation_plan(int rows, int H, int doc_len) {
   return p;
 }
 
-SplitPlan plan_for(int rows, int H, int doc_len, const pp_options* opt) {
-  if (opt && opt->ablation_doc_per_stream) return ablation_plan(rows, H, doc_len);
+SplitPlan plan_for(int rows, int H, int doc_len, const pp_options* opt, bool causal = false) {
+  if (opt && opt->ablation_doc_per_stream && !causal) return ablation_plan(rows, H, doc_len);
   // one slot (a CTA per M tile of a row group) per SM pair by default
   const int ctas = (opt && opt->splits > 0) ? opt->splits
                                            : std::max(1, sm_count() / pp::doc_pair_ctas(rows));
-  return make_plan(rows, H, doc_len, ctas);
+  return make_plan(rows, H, doc_len, ctas, causal);
 }
 
 struct WsLayout {
@@ -118,19 +124,22 @@ long long wait_limit(const pp_options* opt) {
 }
 
 // Shared body of decode and prefill attention.
+// causal: a document prefill; rows = doc_len document tokens, no stream ids.
 pp_status attend(const pp_kv_layer* L, int32_t doc_len, const uint16_t* q, const int16_t* q_sid,
                  const int32_t* q_pos, int32_t rows, float scale, uint16_t* o, float* lse, void* ws,
-                 size_t ws_bytes, const pp_options* opt, void* stream) {
+                 size_t ws_bytes, const pp_options* opt, void* stream, bool causal = false) {
   pp_status s = check_layer(L);
   if (s != PP_OK) return s;
   if (rows < 0 || doc_len < 0) return PP_ERR_INVALID_ARG;
   if (doc_len > L->doc_cap) return PP_ERR_CAPACITY;
   if (rows == 0) return PP_OK;
-  if (!q || !q_sid || !q_pos || !o || !aligned(q, 16) || !aligned(o, 16) || !aligned(q_sid, 2) ||
-      !aligned(q_pos, 4) || (lse && !aligned(lse, 4)))
+  if (!q || !o || !aligned(q, 16) || !aligned(o, 16) || (lse && !aligned(lse, 4)))
+    return PP_ERR_INVALID_ARG;
+  if (!causal && (!q_sid || !q_pos || !aligned(q_sid, 2) || !aligned(q_pos, 4)))
     return PP_ERR_INVALID_ARG;
   if (!(scale == scale)) return PP_ERR_INVALID_ARG;
-  const SplitPlan plan = plan_for(rows, L->H, doc_len, opt);
+  if (causal && opt && opt->ablation_doc_per_stream) return PP_ERR_UNSUPPORTED;
+  const SplitPlan plan = plan_for(rows, L->H, doc_len, opt, causal);
   const bool has_doc = doc_len > 0;
   if (has_doc && plan.C < 1) return PP_ERR_CUDA;  // no device to size the split for
   const WsLayout w = ws_layout(plan, L->d);
@@ -168,11 +177,29 @@ pp_status attend(const pp_kv_layer* L, int32_t doc_len, const uint16_t* q, const
   return from_cuda(mark(2));
 }
 
-size_t workspace(int32_t rows, int32_t H, int32_t d, int32_t doc_len, const pp_options* opt) {
+size_t workspace(int32_t rows, int32_t H, int32_t d, int32_t doc_len, const pp_options* opt,
+                 bool causal = false) {
   if (rows < 0 || H < 1 || (d != 64 && d != 128) || doc_len < 0) return 0;
-  const SplitPlan plan = plan_for(rows, H, doc_len, opt);
+  const SplitPlan plan = plan_for(rows, H, doc_len, opt, causal);
   if (doc_len > 0 && plan.C < 1) return 0;
   return ws_layout(plan, d).total;
+}
+
+// Host copy of a plan for the split-plan test aids.
+pp_status write_plan(const SplitPlan& p, int64_t* h_out, int32_t h_out_len) {
+  if (h_out_len < 5 + 2 * (int64_t)p.units) return PP_ERR_CAPACITY;
+  h_out[0] = p.T;
+  h_out[1] = p.units;
+  h_out[2] = p.W;
+  h_out[3] = p.C;
+  h_out[4] = p.max_chunks;
+  for (int u = 0; u < p.units; ++u) {
+    h_out[5 + 2 * u] = p.W ? pp::plan_cta_of(p, pp::plan_unit_begin(p, u)) : 0;
+    h_out[6 + 2 * u] =
+        p.W ? pp::plan_cta_of(p, pp::plan_unit_begin(p, u) + pp::plan_unit_tiles(p, u % p.G) - 1)
+            : -1;
+  }
+  return PP_OK;
 }
 
 }  // namespace
@@ -238,6 +265,18 @@ PP_API pp_status pp_prefill_attn(const pp_kv_layer* layer, int32_t doc_len, cons
   return attend(layer, doc_len, q, q_sid, q_pos, R, scale, o, lse, ws, ws_bytes, opt, stream);
 }
 
+PP_API size_t pp_doc_prefill_workspace_bytes(int32_t H, int32_t d, int32_t doc_len,
+                                             const pp_options* opt) {
+  return workspace(doc_len, H, d, doc_len, opt, true);
+}
+
+PP_API pp_status pp_doc_prefill_attn(const pp_kv_layer* layer, int32_t doc_len, const uint16_t* q,
+                                     float scale, uint16_t* o, float* lse, void* ws,
+                                     size_t ws_bytes, const pp_options* opt, void* stream) {
+  return attend(layer, doc_len, q, nullptr, nullptr, doc_len, scale, o, lse, ws, ws_bytes, opt,
+                stream, true);
+}
+
 PP_API pp_status pp_debug_visibility(const pp_kv_layer* layer, int32_t doc_len, const int16_t* q_sid,
                               const int32_t* q_pos, int32_t nq, int32_t* count_out,
                               uint8_t* mask_out, void* stream) {
@@ -254,19 +293,15 @@ PP_API pp_status pp_debug_visibility(const pp_kv_layer* layer, int32_t doc_len, 
 PP_API pp_status pp_debug_split_plan(int32_t rows, int32_t H, int32_t doc_len, int32_t ctas,
                               int64_t* h_out, int32_t h_out_len) {
   if (rows < 0 || H < 1 || doc_len < 0 || ctas < 1 || !h_out) return PP_ERR_INVALID_ARG;
-  const SplitPlan p = make_plan(rows, H, doc_len, ctas);
-  if (h_out_len < 5 + 2 * (int64_t)p.units) return PP_ERR_CAPACITY;
-  h_out[0] = p.T;
-  h_out[1] = p.units;
-  h_out[2] = p.W;
-  h_out[3] = p.C;
-  h_out[4] = p.max_chunks;
-  for (int u = 0; u < p.units; ++u) {
-    h_out[5 + 2 * u] = p.W ? pp::plan_cta_of(p, (int64_t)u * p.T) : 0;
-    h_out[6 + 2 * u] = p.W ? pp::plan_cta_of(p, (int64_t)u * p.T + p.T - 1) : -1;
-  }
-  return PP_OK;
+  return write_plan(make_plan(rows, H, doc_len, ctas), h_out, h_out_len);
 }
+
+PP_API pp_status pp_debug_split_plan_causal(int32_t doc_len, int32_t H, int32_t ctas,
+                                            int64_t* h_out, int32_t h_out_len) {
+  if (H < 1 || doc_len < 0 || ctas < 1 || !h_out) return PP_ERR_INVALID_ARG;
+  return write_plan(make_plan(doc_len, H, doc_len, ctas, true), h_out, h_out_len);
+}
+
 
 PP_API pp_status pp_debug_exp2(const float* x, float* y_poly, float* y_hw, int32_t n,
                                void* stream) {

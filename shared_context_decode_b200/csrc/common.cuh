@@ -140,11 +140,46 @@ __device__ __forceinline__ float2 ex2_poly2(float2 x) {
 // u).  Host and device evaluate the same integer formulas.
 struct SplitPlan {
   int64_t W;        // total tiles
-  int32_t C;        // CTAs
-  int32_t T;        // tiles per unit
-  int32_t units;    // H * groups
+  int32_t C;        // slots
+  int32_t T;        // document tiles (a unit's tiles unless causal)
+  int32_t units;    // H * G, unit u = head * G + group (head-major)
   int32_t max_chunks;
+  int32_t G;        // row groups
+  int32_t causal;   // document prefill: row r is document token r and sees keys 0..r,
+                    // so unit (h, g) holds only tiles 0 .. min(T, 2g + 2) - 1
 };
+
+// Tiles of a unit of row group g.
+__host__ __device__ __forceinline__ int32_t plan_unit_tiles(const SplitPlan& p, int g) {
+  return p.causal ? (2 * g + 2 < p.T ? 2 * g + 2 : p.T) : p.T;
+}
+// Tiles of all units of one head: sum over g of plan_unit_tiles (causal:
+// 2g + 2 for every group but the last, which holds T).
+__host__ __device__ __forceinline__ int64_t plan_head_tiles(const SplitPlan& p) {
+  return p.causal ? (int64_t)(p.G - 1) * p.G + p.T : (int64_t)p.G * p.T;
+}
+// First tile of unit u.
+__host__ __device__ __forceinline__ int64_t plan_unit_begin(const SplitPlan& p, int u) {
+  const int h = u / p.G, g = u - h * p.G;
+  return (int64_t)h * plan_head_tiles(p) + (p.causal ? (int64_t)g * (g + 1) : (int64_t)g * p.T);
+}
+// Unit and tile index of global tile t.
+__host__ __device__ __forceinline__ void plan_locate(const SplitPlan& p, int64_t t, int& u, int& j) {
+  const int64_t S = plan_head_tiles(p);
+  const int h = (int)(t / S);
+  const int64_t r = t - (int64_t)h * S;
+  int g;
+  if (p.causal) {  // largest g with g (g + 1) <= r
+    g = (int)((sqrt(4.0 * (double)r + 1.0) - 1.0) * 0.5);
+    while ((int64_t)(g + 1) * (g + 2) <= r) ++g;
+    while (g > 0 && (int64_t)g * (g + 1) > r) --g;
+    if (g > p.G - 1) g = p.G - 1;
+  } else {
+    g = (int)(r / p.T);
+  }
+  u = h * p.G + g;
+  j = (int)(r - (p.causal ? (int64_t)g * (g + 1) : (int64_t)g * p.T));
+}
 
 __host__ __device__ __forceinline__ int64_t plan_tile_begin(const SplitPlan& p, int64_t c) {
   return (c * p.W) / p.C;

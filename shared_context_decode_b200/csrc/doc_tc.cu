@@ -54,7 +54,6 @@ static_assert(128 * kRegsLow + 256 * kRegsHigh <= kThreads * kRegsLaunch, "regis
 struct DocTcParams {
   int rows;
   int H;
-  int G;        // row groups of kGroupRows
   int pair;     // CTAs per slot: 2 when some row group has two M tiles, else 1
   int doc_len;
   SplitPlan plan;
@@ -115,16 +114,18 @@ struct Seg {
 __device__ __forceinline__ bool next_seg(const DocTcParams& p, int64_t& t, int64_t t_end, int slot,
                                          int mt, Seg& s) {
   if (t >= t_end) return false;
-  const int T = p.plan.T;
-  s.u = (int)(t / T);
-  s.j0 = (int)(t - (int64_t)s.u * T);
-  const int64_t ue = (int64_t)s.u * T + T;
-  s.j1 = (int)((ue < t_end ? ue : t_end) - (int64_t)s.u * T);
-  s.h = s.u / p.G;   // unit u = head * G + group (head-major)
-  s.g = s.u - s.h * p.G;
-  s.chunk = slot - plan_cta_of(p.plan, (int64_t)s.u * T);
+  int u, j;
+  plan_locate(p.plan, t, u, j);
+  s.u = u;
+  s.j0 = j;
+  s.h = u / p.plan.G;   // unit u = head * G + group (head-major)
+  s.g = u - s.h * p.plan.G;
+  const int64_t ub = plan_unit_begin(p.plan, u);
+  const int64_t ue = ub + plan_unit_tiles(p.plan, s.g);
+  s.j1 = (int)((ue < t_end ? ue : t_end) - ub);
+  s.chunk = slot - plan_cta_of(p.plan, ub);
   s.active = s.g * kGroupRows + mt * 128 < p.rows;
-  t = (int64_t)s.u * T + s.j1;
+  t = ub + s.j1;
   return true;
 }
 
@@ -462,7 +463,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int c = 0; c < 2; ++c) tmem_ld32(t_S + hf * HB + c * 32, r[c]);
         tmem_ld_wait();
-        const int kvalid = p.doc_len - j * kBN - hf * HB;  // keys of this half inside the document
+        // keys of this half inside the document (and, for a document
+        // prefill, at or before this row's position = its row index)
+        int kvalid = p.doc_len - j * kBN - hf * HB;
+        if (p.plan.causal) {
+          const int krow = s.g * kGroupRows + mt * 128 + rt - (j * kBN + hf * HB) + 1;
+          kvalid = krow < kvalid ? krow : kvalid;
+        }
         if (kvalid < HB) {
 #pragma unroll
           for (int c = 0; c < 2; ++c)
@@ -496,7 +503,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         // P = 2^(S * scale*log2e - m) as bf16 pairs, written over the S
         // buffer's first 64 columns (this half's 32 of them).
-        const float2 sl2v = make_float2(p.sl2, p.sl2), negm = make_float2(-m, -m);
+        // (a row that has seen no key yet keeps m = -inf: its P is 0)
+        const float mneg = m == -INFINITY ? 0.f : -m;
+        const float2 sl2v = make_float2(p.sl2, p.sl2), negm = make_float2(mneg, mneg);
         float2 rs[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
@@ -654,7 +663,6 @@ cudaError_t launch_impl(const pp_kv_layer& L, int doc_len, const uint16_t* q, in
   DocTcParams prm;
   prm.rows = rows;
   prm.H = L.H;
-  prm.G = (rows + kGroupRows - 1) / kGroupRows;
   prm.pair = doc_pair_ctas(rows);
   prm.doc_len = doc_len;
   prm.plan = plan;

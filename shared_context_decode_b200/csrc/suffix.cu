@@ -25,7 +25,8 @@
 //   lse = (M + log2 Lsum) ln 2,
 // the softmax over the union of the key sets in max-shifted form.  Rows that
 // are not answer-stream queries, and rows that see nothing, get o = 0 and
-// lse = -inf.
+// lse = -inf.  Called without stream ids (a document prefill), every row is a
+// document token: no segment keys, only its document partials.
 #include <atomic>
 
 #include "common.cuh"
@@ -162,6 +163,9 @@ __global__ void __launch_bounds__(SufCfg<D>::WARPS * 32) suffix_merge(const SufP
   const int64_t GW = (int64_t)gridDim.x * C::WARPS;
   const int64_t i_begin = gw * items / GW, i_end = (gw + 1) * items / GW;
   const int groups = (p.rows + kGroupRows - 1) / kGroupRows;
+  // document prefill: no stream ids; row r is document token r and sees only
+  // the document (its partials carry the causal mask)
+  const bool doc_rows = p.q_sid == nullptr;
   const size_t seg_elems = (size_t)p.S_cap * D;
 
   uint32_t issued = 0, consumed = 0;
@@ -172,9 +176,9 @@ __global__ void __launch_bounds__(SufCfg<D>::WARPS * 32) suffix_merge(const SufP
     // dependent chain per item
     for (int k = lane; k < cnt; k += 32) {
       const int r = (int)((r0 + k) % p.rows);
-      const int s = p.q_sid[r];
+      const int s = doc_rows ? 0 : p.q_sid[r];
       ItemRec rec;
-      rec.qp = p.q_pos[r];
+      rec.qp = doc_rows ? r : p.q_pos[r];
       rec.s = stream_query(s, p.P_max) ? s : 0;
       rec.n = 0;
       rec.raw = s;
@@ -245,7 +249,7 @@ __global__ void __launch_bounds__(SufCfg<D>::WARPS * 32) suffix_merge(const SufP
       // this lane's key tags, loaded one chunk ahead of their use
       int nsid = sid0, npos = pos0;
       if (k + 1 < cnt) prefetch_item(k + 1);
-      const bool valid = rec.s != 0;
+      const bool valid = rec.s != 0 || doc_rows;
       // document partials of this (row, head), fetched now so their latency
       // hides behind the segment's chunks
       int c0 = 0, c1 = -1;
@@ -253,8 +257,9 @@ __global__ void __launch_bounds__(SufCfg<D>::WARPS * 32) suffix_merge(const SufP
       const int rr = r % kGroupRows;
       if (valid && p.has_doc) {
         const int u = h * groups + r / kGroupRows;
-        c0 = plan_cta_of(p.plan, (int64_t)u * p.plan.T);
-        c1 = plan_cta_of(p.plan, (int64_t)u * p.plan.T + p.plan.T - 1);
+        const int64_t ub = plan_unit_begin(p.plan, u);
+        c0 = plan_cta_of(p.plan, ub);
+        c1 = plan_cta_of(p.plan, ub + plan_unit_tiles(p.plan, r / kGroupRows) - 1);
         slot0 = (int64_t)u * p.plan.max_chunks;
       }
       float2 pre_ml[C::PRE];
@@ -429,7 +434,8 @@ __global__ void __launch_bounds__(SufCfg<D>::WARPS * 32) suffix_merge(const SufP
       }
       if (lane == 0) {
         if (p.lse) p.lse[(int64_t)r * p.H + h] = any ? (m + log2f(l)) * kLn2 : -INFINITY;
-        if (h == 0 && (rec.raw == 0 || rec.raw > p.P_max)) set_status(p.status, PP_DEV_BAD_STREAM);
+        if (h == 0 && !doc_rows && (rec.raw == 0 || rec.raw > p.P_max))
+          set_status(p.status, PP_DEV_BAD_STREAM);
       }
     }
     __syncwarp();

@@ -91,11 +91,17 @@ _exp2 = _sig("pp_debug_exp2", _i32, _vp, _vp, _vp, _i32, _vp)
 _dev_status = _sig("pp_get_device_status", _i32, _LP, ctypes.POINTER(_i32), _vp)
 _split_plan = _sig("pp_debug_split_plan", _i32, _i32, _i32, _i32, _i32,
                    ctypes.POINTER(ctypes.c_int64), _i32)
+_split_plan_causal = _sig("pp_debug_split_plan_causal", _i32, _i32, _i32, _i32,
+                          ctypes.POINTER(ctypes.c_int64), _i32)
+_doc_ws = _sig("pp_doc_prefill_workspace_bytes", _sz, _i32, _i32, _i32, _OP)
+_doc_prefill = _sig("pp_doc_prefill_attn", _i32, _LP, _i32, _vp, ctypes.c_float, _vp, _vp, _vp,
+                    _sz, _OP, _vp)
 
 EXPORTED = ("pp_status_str", "pp_abi_version", "pp_kv_reset", "pp_kv_append",
             "pp_decode_workspace_bytes", "pp_prefill_workspace_bytes", "pp_decode_attn",
             "pp_prefill_attn", "pp_debug_visibility", "pp_get_device_status",
-            "pp_debug_split_plan", "pp_debug_exp2", "pp_decode_attn_noalloc")
+            "pp_debug_split_plan", "pp_debug_exp2", "pp_decode_attn_noalloc",
+            "pp_doc_prefill_workspace_bytes", "pp_doc_prefill_attn", "pp_debug_split_plan_causal")
 
 # Size of the scratch array built into the library for pp_decode_attn_noalloc.
 NOALLOC_SCRATCH_BYTES = 32 << 20
@@ -246,6 +252,33 @@ def _attn(fn, name, layer, doc_len, q, q_sid, q_pos, scale, o, lse, ws, opt, ws_
     return o
 
 
+def doc_prefill_workspace_bytes(H: int, d: int, doc_len: int, opt: Optional[Options] = None):
+    return int(_doc_ws(H, d, doc_len, _opts(opt)))
+
+
+def doc_prefill_attn(layer: KVLayer, doc_len: int, q: torch.Tensor, scale: float,
+                     o: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                     ws: Optional[torch.Tensor] = None,
+                     opt: Optional[Options] = None) -> torch.Tensor:
+    """Causal attention of the document's own tokens: q [doc_len, H, d] bf16,
+    row i = document token i; its K/V must already be appended (stream 0)."""
+    dev = layer.device
+    _want(q, torch.bfloat16, "q", dev)
+    if q.shape != (doc_len, layer.H, layer.d):
+        raise ValueError("pp_doc_prefill_attn: q must be [doc_len, H, d]")
+    if o is None:
+        o = torch.empty_like(q)
+    _want(o, torch.bfloat16, "o", dev)
+    if lse is not None:
+        _want(lse, torch.float32, "lse", dev)
+    if ws is None:
+        ws = workspace(doc_prefill_workspace_bytes(layer.H, layer.d, doc_len, opt), dev)
+    _want(ws, torch.uint8, "ws", dev)
+    _check(_doc_prefill(layer.ref, doc_len, _ptr(q), float(scale), _ptr(o), _ptr(lse), _ptr(ws),
+                        ws.numel(), _opts(opt), _stream(dev)), "pp_doc_prefill_attn")
+    return o
+
+
 def decode_attn(layer: KVLayer, doc_len: int, q: torch.Tensor, q_sid: torch.Tensor,
                 q_pos: torch.Tensor, scale: float, o: Optional[torch.Tensor] = None,
                 lse: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
@@ -322,12 +355,16 @@ def device_status(layer: KVLayer) -> int:
     return int(out.value)
 
 
-def split_plan(rows: int, H: int, doc_len: int, ctas: int):
+def split_plan(rows: int, H: int, doc_len: int, ctas: int, causal: bool = False):
     """The document split the library would use: dict with T, units, W, C,
-    max_chunks and, per unit, its (first CTA, last CTA)."""
-    units = -(-rows // 256) * H
+    max_chunks and, per unit, its (first CTA, last CTA).  causal: the split
+    of a document prefill (rows = doc_len)."""
+    units = -(-(doc_len if causal else rows) // 256) * H
     buf = (ctypes.c_int64 * (5 + 2 * units))()
-    _check(_split_plan(rows, H, doc_len, ctas, buf, len(buf)), "pp_debug_split_plan")
+    if causal:
+        _check(_split_plan_causal(doc_len, H, ctas, buf, len(buf)), "pp_debug_split_plan_causal")
+    else:
+        _check(_split_plan(rows, H, doc_len, ctas, buf, len(buf)), "pp_debug_split_plan")
     vals = list(buf)
     return dict(T=vals[0], units=vals[1], W=vals[2], C=vals[3], max_chunks=vals[4],
                 chunks=[(vals[5 + 2 * u], vals[6 + 2 * u]) for u in range(units)])

@@ -123,3 +123,53 @@ def test_split_plan_invariants(pp, rows, H, doc_len, ctas):
         assert (c0, c1) == (meets[0], meets[-1])
         assert c1 - c0 + 1 <= p["max_chunks"]
     assert p["max_chunks"] == max(c1 - c0 + 1 for c0, c1 in p["chunks"])
+
+
+@pytest.mark.parametrize("doc_len,H,ctas", [
+    (16384, 32, 74), (12000, 4, 148), (1000, 3, 7), (300, 2, 5), (129, 1, 3), (1, 1, 148),
+    (256, 2, 1), (257, 5, 16), (2049, 1, 9)])
+def test_causal_split_plan_invariants(pp, doc_len, H, ctas):
+    """Document prefill split: unit (head, group g) holds key tiles
+    0 .. min(T, 2g+2)-1 (rows 256g..256g+255 see keys up to their own
+    position), units laid out head-major, ranges balanced over the slots."""
+    p = pp.split_plan(doc_len, H, doc_len, ctas, causal=True)
+    T = -(-doc_len // 128)
+    G = -(-doc_len // 256)
+    tiles = [min(T, 2 * g + 2) for g in range(G)]
+    # every key tile a group's rows can see is in its unit, and no more
+    for g in range(G):
+        last_row = min(doc_len, 256 * (g + 1)) - 1
+        assert tiles[g] == last_row // 128 + 1
+    W = H * sum(tiles)
+    assert p["T"] == T and p["units"] == G * H and p["W"] == W
+    C = p["C"]
+    assert C == min(ctas, W)
+    begin = [c * W // C for c in range(C + 1)]
+    ub = 0
+    for u, (c0, c1) in enumerate(p["chunks"]):
+        n = tiles[u % G]
+        meets = [c for c in range(C) if begin[c] < ub + n and begin[c + 1] > ub]
+        assert (c0, c1) == (meets[0], meets[-1])
+        ub += n
+    assert ub == W
+    assert p["max_chunks"] == max(c1 - c0 + 1 for c0, c1 in p["chunks"])
+
+
+def test_doc_prefill_host_validation(pp):
+    L = fake_layer(pp)
+
+    def call(doc_len=10, q=0x90000, ws_bytes=1 << 30, opt=None, o=0xC0000):
+        return pp._doc_prefill(ctypes.byref(L), doc_len, q, 0.1, o, None, 0xD0000, ws_bytes,
+                               None if opt is None else ctypes.byref(opt), None)
+
+    assert call(doc_len=0) == pp.PP_OK                              # nothing to do
+    assert call(doc_len=-1) == pp.PP_ERR_INVALID_ARG
+    assert call(doc_len=1025) == pp.PP_ERR_CAPACITY                # above doc_cap
+    assert call(q=0x90004) == pp.PP_ERR_INVALID_ARG                # misaligned q
+    assert call(o=0) == pp.PP_ERR_INVALID_ARG
+    assert call(opt=pp.Options(ablation_doc_per_stream=1)) == pp.PP_ERR_UNSUPPORTED
+    assert call(ws_bytes=16, opt=pp.Options(splits=4)) == pp.PP_ERR_CAPACITY
+    opt = pp.Options(splits=148)
+    plan = pp.split_plan(5000, 32, 5000, 148, causal=True)
+    slots = plan["units"] * plan["max_chunks"] * 256
+    assert pp.doc_prefill_workspace_bytes(32, 128, 5000, opt) == slots * 128 * 4 + slots * 2 * 4

@@ -290,3 +290,31 @@ def test_append_replay_invariants():
         assert got == sent[s][:S]
         assert R.length(s) == min(len(sent[s]), S)
     assert ("segment_overflow" in R.flags) == any(len(sent[s]) > S for s in sent)
+
+
+def test_document_queries_equal_causal_brute_force():
+    """Document prefill (project page "Read Once, Answer Many", section "How
+    it works": the document is encoded once): a document token (stream 0)
+    attends to the document tokens at or before its position -- ordinary
+    causal attention, checked against the stream-free brute force."""
+    rng = np.random.default_rng(7)
+    N, H, d = 37, 2, 8
+
+    def rbits(shape):   # random values rounded to bf16
+        t = torch.tensor(rng.standard_normal(shape), dtype=torch.float32).to(torch.bfloat16)
+        return t.view(torch.int16).numpy().view(np.uint16)
+
+    k, v, q = rbits((N, H, d)), rbits((N, H, d)), rbits((N, H, d))
+    pos = np.arange(N, dtype=np.int32)
+    # a stream token that no document query may see
+    k2 = np.concatenate([k, rbits((1, H, d))])
+    v2 = np.concatenate([v, f2bits(100.0 * np.ones((1, H, d)))])
+    ks = np.concatenate([np.zeros(N, np.int32), [1]])
+    kp = np.concatenate([pos, [N]])
+    o, lse, nvis = oracle.masked_attention(q, np.zeros(N, np.int32), pos, k2, v2, ks, kp, 0.3)
+    ref_o, ref_lse = brute.causal_attention(brute.bf16_bits_to_f64(q), pos,
+                                            brute.bf16_bits_to_f64(k), brute.bf16_bits_to_f64(v),
+                                            pos, 0.3)
+    np.testing.assert_allclose(o, ref_o, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse, ref_lse, rtol=0, atol=1e-11)
+    assert nvis.tolist() == list(range(1, N + 1))
