@@ -132,6 +132,20 @@ int32_t pp_abi_version(void);
 pp_status pp_kv_reset(const pp_kv_layer *layer, void *stream);
 
 /*
+ * Free the segments of n streams for new questions (continuous batching:
+ * a stream that has finished its answer hands its segment to the next
+ * question of the request).  sid: device int16 [n], stream ids 1..P_max;
+ * each listed stream's len is set to 0, so its old slots are invisible (a
+ * slot is visible only below len) and the next pp_kv_append of that stream
+ * writes from slot 0.  Ids outside 1..P_max set PP_DEV_BAD_STREAM and are
+ * skipped; -1 entries are ignored, so a fixed-shape list can carry unused
+ * places.  Asynchronous, capture-safe.  The pages have no counterpart: their
+ * engine starts a new request for new questions.
+ */
+pp_status pp_kv_reset_streams(const pp_kv_layer *layer, const int16_t *sid, int32_t n,
+                              void *stream);
+
+/*
  * Append n rows to the cache ("How it works": each decode step appends one
  * token per stream; the document is written once as stream 0).
  *   k, v  bf16 [n][H][d];  sid int16 [n];  pos int32 [n].

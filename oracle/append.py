@@ -12,6 +12,10 @@ KV slot carries a stream id; each decode step appends one token per stream):
     (S_cap slots) drops the row and raises 'segment_overflow';
   * a row with stream id < 0 is an inactive row and is skipped silently;
   * a stream id above P_max drops the row and raises 'bad_stream'.
+Refill (continuous batching; the pages have none, this library's rule):
+  * resetting stream s empties its slot list, so its next rows start again
+    at slot 0; id -1 is ignored, any other id outside [1, P_max] raises
+    'bad_stream'.
 """
 import numpy as np
 
@@ -42,6 +46,16 @@ class AppendReplay:
                 self.flags.add("segment_overflow")
                 continue
             self.seg[s].append((np.array(k[i]), np.array(v[i]), s, p))
+
+    def reset_streams(self, sids):
+        for s in sids:
+            s = int(s)
+            if s == -1:
+                continue
+            if not 1 <= s <= self.P_max:
+                self.flags.add("bad_stream")
+                continue
+            self.seg[s] = []
 
     def length(self, s):
         return len(self.seg[s])

@@ -228,6 +228,17 @@ PP_API pp_status pp_kv_reset(const pp_kv_layer* layer, void* stream) {
   return from_cuda(pp::launch_kv_reset(*layer, static_cast<cudaStream_t>(stream)));
 }
 
+PP_API pp_status pp_kv_reset_streams(const pp_kv_layer* layer, const int16_t* sid, int32_t n,
+                                     void* stream) {
+  pp_status s = check_layer(layer);
+  if (s != PP_OK) return s;
+  if (n < 0) return PP_ERR_INVALID_ARG;
+  if (n == 0) return PP_OK;
+  if (!sid || !aligned(sid, 2)) return PP_ERR_INVALID_ARG;
+  return from_cuda(
+      pp::launch_kv_reset_streams(*layer, sid, n, static_cast<cudaStream_t>(stream)));
+}
+
 PP_API pp_status pp_kv_append(const pp_kv_layer* layer, const uint16_t* k, const uint16_t* v,
                        const int16_t* sid, const int32_t* pos, int32_t n, void* stream) {
   pp_status s = check_layer(layer);

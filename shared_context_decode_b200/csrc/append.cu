@@ -93,6 +93,26 @@ __global__ void kv_reset_kernel(pp_kv_layer L) {
   if (blockIdx.x == 0 && threadIdx.x == 0) *L.status = 0;
 }
 
+// Zero len[] of the listed streams (continuous-batching refill).
+__global__ void kv_reset_streams_kernel(pp_kv_layer L, const int16_t* __restrict__ sid, int n) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
+    const int s = sid[i];
+    if (s == -1) continue;
+    if (s < 1 || s > L.P_max) {
+      set_status(L.status, PP_DEV_BAD_STREAM);
+      continue;
+    }
+    L.len[s - 1] = 0;
+  }
+}
+
+cudaError_t launch_kv_reset_streams(const pp_kv_layer& L, const int16_t* sid, int n,
+                                    cudaStream_t st) {
+  const int blocks = (n + 255) / 256 < 148 ? (n + 255) / 256 : 148;
+  kv_reset_streams_kernel<<<blocks, 256, 0, st>>>(L, sid, n);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_kv_append(const pp_kv_layer& L, const uint16_t* k, const uint16_t* v,
                              const int16_t* sid, const int32_t* pos, int n, cudaStream_t st) {
   kv_append_rows<<<n, 128, 0, st>>>(L, reinterpret_cast<const uint4*>(k),

@@ -21,6 +21,8 @@ bool make_tmap_bf16_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d
 cudaError_t launch_kv_append(const pp_kv_layer& L, const uint16_t* k, const uint16_t* v,
                              const int16_t* sid, const int32_t* pos, int n, cudaStream_t st);
 cudaError_t launch_kv_reset(const pp_kv_layer& L, cudaStream_t st);
+cudaError_t launch_kv_reset_streams(const pp_kv_layer& L, const int16_t* sid, int n,
+                                    cudaStream_t st);
 
 // Document pass on the tensor cores; tensor maps are built inside.
 cudaError_t launch_doc_pass_tc(const pp_kv_layer& L, int doc_len, const uint16_t* q, int rows,

@@ -93,6 +93,7 @@ _split_plan = _sig("pp_debug_split_plan", _i32, _i32, _i32, _i32, _i32,
                    ctypes.POINTER(ctypes.c_int64), _i32)
 _split_plan_causal = _sig("pp_debug_split_plan_causal", _i32, _i32, _i32, _i32,
                           ctypes.POINTER(ctypes.c_int64), _i32)
+_reset_streams = _sig("pp_kv_reset_streams", _i32, _LP, _vp, _i32, _vp)
 _doc_ws = _sig("pp_doc_prefill_workspace_bytes", _sz, _i32, _i32, _i32, _OP)
 _doc_prefill = _sig("pp_doc_prefill_attn", _i32, _LP, _i32, _vp, ctypes.c_float, _vp, _vp, _vp,
                     _sz, _OP, _vp)
@@ -101,7 +102,8 @@ EXPORTED = ("pp_status_str", "pp_abi_version", "pp_kv_reset", "pp_kv_append",
             "pp_decode_workspace_bytes", "pp_prefill_workspace_bytes", "pp_decode_attn",
             "pp_prefill_attn", "pp_debug_visibility", "pp_get_device_status",
             "pp_debug_split_plan", "pp_debug_exp2", "pp_decode_attn_noalloc",
-            "pp_doc_prefill_workspace_bytes", "pp_doc_prefill_attn", "pp_debug_split_plan_causal")
+            "pp_doc_prefill_workspace_bytes", "pp_doc_prefill_attn", "pp_debug_split_plan_causal",
+            "pp_kv_reset_streams")
 
 # Size of the scratch array built into the library for pp_decode_attn_noalloc.
 NOALLOC_SCRATCH_BYTES = 32 << 20
@@ -199,6 +201,14 @@ class KVLayer:
 
 def kv_reset(layer: KVLayer):
     _check(_kv_reset(layer.ref, _stream(layer.device)), "pp_kv_reset")
+
+
+def kv_reset_streams(layer: KVLayer, sid: torch.Tensor):
+    """Free the segments of the streams listed in sid [n] int16 (ids 1..P_max,
+    -1 = unused place) for new questions: their len becomes 0."""
+    _want(sid, torch.int16, "sid", layer.device)
+    _check(_reset_streams(layer.ref, _ptr(sid), sid.numel(), _stream(layer.device)),
+           "pp_kv_reset_streams")
 
 
 def kv_append(layer: KVLayer, k: torch.Tensor, v: torch.Tensor, sid: torch.Tensor,

@@ -173,3 +173,12 @@ def test_doc_prefill_host_validation(pp):
     plan = pp.split_plan(5000, 32, 5000, 148, causal=True)
     slots = plan["units"] * plan["max_chunks"] * 256
     assert pp.doc_prefill_workspace_bytes(32, 128, 5000, opt) == slots * 128 * 4 + slots * 2 * 4
+
+
+def test_reset_streams_host_validation(pp):
+    L = fake_layer(pp)
+    assert pp._reset_streams(ctypes.byref(L), 0x1000, 0, None) == pp.PP_OK    # nothing to do
+    assert pp._reset_streams(ctypes.byref(L), 0x1000, -1, None) == pp.PP_ERR_INVALID_ARG
+    assert pp._reset_streams(ctypes.byref(L), None, 3, None) == pp.PP_ERR_INVALID_ARG
+    assert pp._reset_streams(ctypes.byref(L), 0x1001, 3, None) == pp.PP_ERR_INVALID_ARG
+    assert pp._reset_streams(None, 0x1000, 3, None) == pp.PP_ERR_INVALID_ARG

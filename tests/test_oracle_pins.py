@@ -318,3 +318,20 @@ def test_document_queries_equal_causal_brute_force():
     np.testing.assert_allclose(o, ref_o, rtol=0, atol=1e-12)
     np.testing.assert_allclose(lse, ref_lse, rtol=0, atol=1e-11)
     assert nvis.tolist() == list(range(1, N + 1))
+
+
+def test_append_replay_refill_hand_case():
+    """Refill rule by hand: after stream 2 is reset its next row lands in slot
+    0 again, other streams keep their slots, -1 is ignored and an id outside
+    1..P_max raises bad_stream."""
+    R = AppendReplay(3, 4, 8)
+    rows = np.arange(1, 7, dtype=np.int64).reshape(6, 1, 1)
+    R.append(rows, -rows, [1, 2, 2, 3, 2, 1], [10, 10, 11, 10, 12, 11])
+    assert [R.length(s) for s in (1, 2, 3)] == [2, 3, 1]
+    R.reset_streams([2, -1])
+    assert [R.length(s) for s in (1, 2, 3)] == [2, 0, 1] and not R.flags
+    R.append(np.array([[[7]]]), np.array([[[-7]]]), [2], [10])
+    assert [(int(t[0][0, 0]), t[2], t[3]) for t in R.seg[2]] == [(7, 2, 10)]
+    assert [int(t[0][0, 0]) for t in R.seg[1]] == [1, 6]
+    R.reset_streams([4])
+    assert R.flags == {"bad_stream"}
