@@ -26,6 +26,8 @@ Secondary measurements (--mode, one GPU, one JSON line each):
             document part's TFLOP/s
   ablation  the decode step with the per-stream document pass (every stream
             reads the whole document) instead of the shared one
+  siblingscan  the decode step with the suffix part done as the pages' kernel
+            does it (every query scans all streams' answer tokens, masked)
   docprefill  causal attention of a 16384-token document over its own
             tokens (pp_doc_prefill_attn), 32 heads, d = 128; tokens/s and TFLOP/s
   sweep     answer generation over doc x streams: 32 decode steps x 32
@@ -362,25 +364,32 @@ def mode_prefill(args, world, rank, local, dev):
     del step.graph
 
 
-def mode_ablation(args, world, rank, local, dev):
+def mode_ablation(args, world, rank, local, dev, sibling=False):
     from shared_context_decode_b200 import workloads as wl
     nl = args.layers or 4
     step = DecodeStep(args.workload, nl, dev)
     pp = step.pp
-    step.opts = [pp.Options(ablation_doc_per_stream=1) for _ in range(nl)]
+    step.opts = [pp.Options(sibling_scan=1) if sibling else pp.Options(ablation_doc_per_stream=1)
+                 for _ in range(nl)]
     step.capture()
     W = step.W
     ms, clocks = timed_replays(step, args.steps, args.warmup, world, local)
     step.check_status()
     value, ms = aggregate(W.P, ms, world, dev)
     shared_b, _ = doc_pass_algorithmic(W)
-    line = {"mode": "ablation", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+    line = {"mode": "siblingscan" if sibling else "ablation", "metric": METRIC, "value": value,
+            "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
             "config": {"workload": args.workload, "layers": nl, "H": W.H, "d": W.d,
-                       "doc_tokens": W.N, "streams": W.P, "ablation": "doc_per_stream"},
-            "doc_bytes_per_layer_shared": shared_b, "doc_bytes_per_layer_ablation": shared_b * W.P,
+                       "doc_tokens": W.N, "streams": W.P,
+                       "ablation": "sibling_scan" if sibling else "doc_per_stream"},
+            **({"suffix_keys_per_query_scanned": W.suffix_tokens() + W.P,
+                "suffix_keys_per_query_own_segment": (W.suffix_tokens() + W.P) / W.P}
+               if sibling else
+               {"doc_bytes_per_layer_shared": shared_b,
+                "doc_bytes_per_layer_ablation": shared_b * W.P}),
             "gpu_launches": step.kernels_per_step() * args.steps, "clocks": clocks}
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -698,7 +707,7 @@ def main():
     ap.add_argument("--ref-seconds", type=float, default=10.0)
     ap.add_argument("--roofline-reps", type=int, default=3)
     ap.add_argument("--mode", default="decode",
-                    choices=["decode", "prefill", "ablation", "sweep", "docprefill"],
+                    choices=["decode", "prefill", "ablation", "siblingscan", "sweep", "docprefill"],
                     help="decode: the headline step (default); others: secondary measurements")
     args = ap.parse_args()
     world, rank, local = dist_env()
@@ -718,7 +727,8 @@ def main():
     dev = torch.device("cuda", local)
     if args.mode != "decode":
         {"prefill": mode_prefill, "ablation": mode_ablation, "sweep": mode_sweep,
-         "docprefill": mode_docprefill}[args.mode](
+         "docprefill": mode_docprefill,
+         "siblingscan": lambda *a: mode_ablation(*a, sibling=True)}[args.mode](
             args, world, rank, local, dev)
         if world > 1:
             import torch.distributed as dist

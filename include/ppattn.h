@@ -113,6 +113,12 @@ typedef struct pp_kv_layer {
  *                           events; the work done is unchanged).  During a
  *                           stream capture they are recorded as external
  *                           event-record nodes, i.e. at every graph replay.
+ *   sibling_scan            1 = the suffix part as the pages' kernel does it:
+ *                           every query scans the answer tokens of ALL
+ *                           streams and the stream mask rejects the siblings'
+ *                           (project page, section "More results"); same
+ *                           result, kept to measure what per-stream segments
+ *                           save.  Decode and question prefill only.
  */
 typedef struct pp_options {
     int32_t splits;
@@ -120,6 +126,7 @@ typedef struct pp_options {
     int32_t debug_inject_timeout;
     int32_t wait_limit_log2;
     void **events;
+    int32_t sibling_scan;
 } pp_options;
 
 /* Human-readable name of a pp_status value. */

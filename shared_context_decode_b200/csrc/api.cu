@@ -138,7 +138,8 @@ pp_status attend(const pp_kv_layer* L, int32_t doc_len, const uint16_t* q, const
   if (!causal && (!q_sid || !q_pos || !aligned(q_sid, 2) || !aligned(q_pos, 4)))
     return PP_ERR_INVALID_ARG;
   if (!(scale == scale)) return PP_ERR_INVALID_ARG;
-  if (causal && opt && opt->ablation_doc_per_stream) return PP_ERR_UNSUPPORTED;
+  if (causal && opt && (opt->ablation_doc_per_stream || opt->sibling_scan))
+    return PP_ERR_UNSUPPORTED;
   const SplitPlan plan = plan_for(rows, L->H, doc_len, opt, causal);
   const bool has_doc = doc_len > 0;
   if (has_doc && plan.C < 1) return PP_ERR_CUDA;  // no device to size the split for
@@ -171,9 +172,15 @@ pp_status attend(const pp_kv_layer* L, int32_t doc_len, const uint16_t* q, const
     if (e != cudaSuccess) return PP_ERR_CUDA;
   }
   if (mark(1) != cudaSuccess) return PP_ERR_CUDA;
-  if ((s = from_cuda(pp::launch_suffix_merge(*L, q, q_sid, q_pos, rows, scale, plan, has_doc, part,
-                                             o, lse, wait_limit(opt), sms, st))) != PP_OK)
+  if (opt && opt->sibling_scan) {
+    if ((s = from_cuda(pp::launch_sibling_scan(*L, q, q_sid, q_pos, rows, scale, plan, has_doc,
+                                               part, o, lse, st))) != PP_OK)
+      return s;
+  } else if ((s = from_cuda(pp::launch_suffix_merge(*L, q, q_sid, q_pos, rows, scale, plan,
+                                                    has_doc, part, o, lse, wait_limit(opt), sms,
+                                                    st))) != PP_OK) {
     return s;
+  }
   return from_cuda(mark(2));
 }
 

@@ -31,6 +31,12 @@ cudaError_t launch_doc_pass_tc(const pp_kv_layer& L, int doc_len, const uint16_t
 cudaError_t launch_doc_per_stream(const pp_kv_layer& L, int doc_len, const uint16_t* q, int rows,
                                   float scale, int max_chunks, const Partials& part,
                                   cudaStream_t st);
+// Comparison mode: every query scans all streams' segments (masked), then
+// the merge; writes o and lse.
+cudaError_t launch_sibling_scan(const pp_kv_layer& L, const uint16_t* q, const int16_t* q_sid,
+                                const int32_t* q_pos, int rows, float scale, const SplitPlan& plan,
+                                bool has_doc, const Partials& part, uint16_t* o, float* lse,
+                                cudaStream_t st);
 // Suffix pass with the log-sum-exp merge in its epilogue; writes o and lse.
 cudaError_t launch_suffix_merge(const pp_kv_layer& L, const uint16_t* q, const int16_t* q_sid,
                                 const int32_t* q_pos, int rows, float scale, const SplitPlan& plan,

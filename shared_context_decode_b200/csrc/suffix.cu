@@ -605,4 +605,157 @@ cudaError_t launch_doc_per_stream(const pp_kv_layer& L, int doc_len, const uint1
   return cudaGetLastError();
 }
 
+// Sibling scan (comparison mode): the suffix part as the pages' kernel does
+// it -- every query scans the answer tokens of ALL streams and the stream
+// mask rejects the siblings' ("Read Once, Answer Many" project page,
+// section "More results": the kernel scans its sibling streams' answer
+// tokens, so its cost grows with the number of streams).  One warp per
+// (row, head) over every segment of head h, CUDA cores, the same mask
+// predicate; then the merge with the document partials as in suffix_merge.
+// Reads sum_s len[s] keys per item instead of len[own stream].
+template <int D>
+__global__ void __launch_bounds__(256) sibling_scan(pp_kv_layer L, const uint16_t* __restrict__ q,
+                                                    const int16_t* __restrict__ q_sid,
+                                                    const int32_t* __restrict__ q_pos, int rows,
+                                                    float sl2, SplitPlan plan, int has_doc,
+                                                    const float* __restrict__ doc_o,
+                                                    const float* __restrict__ doc_ml,
+                                                    uint16_t* __restrict__ o,
+                                                    float* __restrict__ lse) {
+  constexpr int LPK = D / 8, KPI = 32 / LPK, U = 4;
+  const int64_t w = (int64_t)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
+  if (w >= (int64_t)rows * L.H) return;
+  const int h = (int)(w / rows), r = (int)(w - (int64_t)h * rows);
+  const int lane = threadIdx.x & 31, g = lane / LPK, j = lane % LPK;
+  const int raw = q_sid[r];
+  const int s = stream_query(raw, L.P_max) ? raw : 0;
+  const int qp = q_pos[r];
+  float m = -INFINITY, l = 0.f, acc[8];
+#pragma unroll
+  for (int c = 0; c < 8; ++c) acc[c] = 0.f;
+  if (s) {
+    const uint4 qv = reinterpret_cast<const uint4*>(q + ((int64_t)r * L.H + h) * D)[j];
+    float qf[8];
+    {
+      const uint32_t wq[4] = {qv.x, qv.y, qv.z, qv.w};
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const float2 f = bf2_to_f2(wq[c]);
+        qf[2 * c] = f.x * sl2;
+        qf[2 * c + 1] = f.y * sl2;
+      }
+    }
+    for (int s2 = 1; s2 <= L.P_max; ++s2) {
+      const int n = min(L.len[s2 - 1], L.S_cap);
+      const size_t seg = ((size_t)(s2 - 1) * L.H + h) * L.S_cap;
+      const uint4* kb = reinterpret_cast<const uint4*>(L.k_suf) + seg * LPK;
+      const uint4* vb = reinterpret_cast<const uint4*>(L.v_suf) + seg * LPK;
+      const int16_t* sb = L.sid + (size_t)(s2 - 1) * L.S_cap;
+      const int32_t* pb = L.pos + (size_t)(s2 - 1) * L.S_cap;
+      for (int t0 = 0; t0 < n; t0 += KPI * U) {
+        uint4 kk[U], vv[U];
+        bool vis[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          const int t = t0 + u * KPI + g;
+          vis[u] = t < n && slot_visible(s, qp, sb[t], pb[t], t, n);
+          if (t < n) {
+            kk[u] = kb[(int64_t)t * LPK + j];
+            vv[u] = vb[(int64_t)t * LPK + j];
+          }
+        }
+        float x[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          float dot = 0.f;
+          if (t0 + u * KPI < n) {
+            const uint32_t wk[4] = {kk[u].x, kk[u].y, kk[u].z, kk[u].w};
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              const float2 f = bf2_to_f2(wk[c]);
+              dot = fmaf(qf[2 * c], f.x, dot);
+              dot = fmaf(qf[2 * c + 1], f.y, dot);
+            }
+#pragma unroll
+            for (int o2 = 1; o2 < LPK; o2 <<= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o2);
+          }
+          x[u] = vis[u] ? dot : -INFINITY;
+        }
+        float cm = m;
+#pragma unroll
+        for (int u = 0; u < U; ++u) cm = fmaxf(cm, x[u]);
+        if (cm == -INFINITY) continue;
+        const float corr = exp2f(m - cm);
+        l *= corr;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) acc[c] *= corr;
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          if (x[u] == -INFINITY) continue;
+          const float pr = exp2f(x[u] - cm);
+          l += pr;
+          const uint32_t wv[4] = {vv[u].x, vv[u].y, vv[u].z, vv[u].w};
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const float2 f = bf2_to_f2(wv[c]);
+            acc[2 * c] = fmaf(pr, f.x, acc[2 * c]);
+            acc[2 * c + 1] = fmaf(pr, f.y, acc[2 * c + 1]);
+          }
+        }
+        m = cm;
+      }
+    }
+    combine_groups<LPK>(m, l, acc);
+    // merge with the document partials of (row, head)
+    if (has_doc) {
+      const int groups = (rows + kGroupRows - 1) / kGroupRows;
+      const int u = h * groups + r / kGroupRows;
+      const int64_t ub = plan_unit_begin(plan, u);
+      const int c0 = plan_cta_of(plan, ub);
+      const int c1 = plan_cta_of(plan, ub + plan_unit_tiles(plan, r / kGroupRows) - 1);
+      const int64_t slot0 = (int64_t)u * plan.max_chunks;
+      for (int c = c0; c <= c1; ++c) {
+        const int64_t sl = (slot0 + c - c0) * kGroupRows + r % kGroupRows;
+        const float2 ml = reinterpret_cast<const float2*>(doc_ml)[sl];
+        float a2[8];
+        const float4* src = reinterpret_cast<const float4*>(doc_o + sl * D + j * 8);
+        const float4 v0 = src[0], v1 = src[1];
+        a2[0] = v0.x; a2[1] = v0.y; a2[2] = v0.z; a2[3] = v0.w;
+        a2[4] = v1.x; a2[5] = v1.y; a2[6] = v1.z; a2[7] = v1.w;
+        fold(m, l, acc, ml.x, ml.y, a2);
+      }
+    }
+  }
+  const bool any = s != 0 && l > 0.f;
+  const float inv = any ? 1.f / l : 0.f;
+  if (g == 0) {
+    uint4 pk;
+    pk.x = f2_to_bf2(acc[0] * inv, acc[1] * inv);
+    pk.y = f2_to_bf2(acc[2] * inv, acc[3] * inv);
+    pk.z = f2_to_bf2(acc[4] * inv, acc[5] * inv);
+    pk.w = f2_to_bf2(acc[6] * inv, acc[7] * inv);
+    reinterpret_cast<uint4*>(o + ((int64_t)r * L.H + h) * D)[j] = pk;
+  }
+  if (lane == 0) {
+    if (lse) lse[(int64_t)r * L.H + h] = any ? (m + log2f(l)) * kLn2 : -INFINITY;
+    if (h == 0 && (raw == 0 || raw > L.P_max)) set_status(L.status, PP_DEV_BAD_STREAM);
+  }
+}
+
+cudaError_t launch_sibling_scan(const pp_kv_layer& L, const uint16_t* q, const int16_t* q_sid,
+                                const int32_t* q_pos, int rows, float scale, const SplitPlan& plan,
+                                bool has_doc, const Partials& part, uint16_t* o, float* lse,
+                                cudaStream_t st) {
+  const int64_t warps = (int64_t)rows * L.H;
+  const int blocks = (int)((warps + 7) / 8);
+  const float sl2 = scale * kLog2e;
+  if (L.d == 128)
+    sibling_scan<128><<<blocks, 256, 0, st>>>(L, q, q_sid, q_pos, rows, sl2, plan, has_doc ? 1 : 0,
+                                              part.doc_o, part.doc_ml, o, lse);
+  else
+    sibling_scan<64><<<blocks, 256, 0, st>>>(L, q, q_sid, q_pos, rows, sl2, plan, has_doc ? 1 : 0,
+                                             part.doc_o, part.doc_ml, o, lse);
+  return cudaGetLastError();
+}
+
 }  // namespace pp

@@ -168,6 +168,7 @@ def test_doc_prefill_host_validation(pp):
     assert call(q=0x90004) == pp.PP_ERR_INVALID_ARG                # misaligned q
     assert call(o=0) == pp.PP_ERR_INVALID_ARG
     assert call(opt=pp.Options(ablation_doc_per_stream=1)) == pp.PP_ERR_UNSUPPORTED
+    assert call(opt=pp.Options(sibling_scan=1)) == pp.PP_ERR_UNSUPPORTED
     assert call(ws_bytes=16, opt=pp.Options(splits=4)) == pp.PP_ERR_CAPACITY
     opt = pp.Options(splits=148)
     plan = pp.split_plan(5000, 32, 5000, 148, causal=True)
