@@ -168,6 +168,7 @@ __global__ void __launch_bounds__(SufCfg<D>::WARPS * 32) suffix_merge(const SufP
   const bool doc_rows = p.q_sid == nullptr;
   const size_t seg_elems = (size_t)p.S_cap * D;
 
+  const uint64_t pol_first = l2_policy_evict_first();
   uint32_t issued = 0, consumed = 0;
   bool ok = true;
   for (int64_t r0 = i_begin; ok && r0 < i_end; r0 += C::TBL) {
@@ -210,8 +211,10 @@ __global__ void __launch_bounds__(SufCfg<D>::WARPS * 32) suffix_merge(const SufP
         uint8_t* st = ring + stage * C::STAGE;
         fence_proxy_async();
         mbar_arrive_expect_tx(full + stage, 2u * nk * C::ROWB);
-        bulk_load(st, p.k_suf + seg, nk * C::ROWB, full + stage);
-        bulk_load(st + C::HALF, p.v_suf + seg, nk * C::ROWB, full + stage);
+        // evict-first: the rows are read once; the document partials the
+        // merge reads next stay in L2
+        bulk_load_hint(st, p.k_suf + seg, nk * C::ROWB, full + stage, pol_first);
+        bulk_load_hint(st + C::HALF, p.v_suf + seg, nk * C::ROWB, full + stage, pol_first);
       }
       pt0 += C::CK;
       return true;
