@@ -301,14 +301,14 @@ class PrefillStep:
         self.ws = pp.workspace(pp.prefill_workspace_bytes(W.R, W.H, W.d, W.N), device)
         self.graph = None
 
-    def run_eager(self):
+    def run_eager(self, opts=None):
         pp = self.pp
         self.len_all.zero_()
         for l in range(self.layers):
             x = self.inp[l]
             pp.kv_append(self.cache[l], x["k"], x["v"], x["sid"], x["pos"])
             pp.prefill_attn(self.cache[l], self.W.N, x["q"], x["sid"], x["pos"], self.W.scale,
-                            o=x["o"], ws=self.ws)
+                            o=x["o"], ws=self.ws, opt=None if opts is None else opts[l])
 
     capture = DecodeStep.capture
     replay = DecodeStep.replay
@@ -350,6 +350,8 @@ def mode_prefill(args, world, rank, local, dev):
     flops = 4.0 * W.R * W.N * W.d * W.H * nl
     tfs = flops / (ms / 1e3) / 1e12 * world
     peaks = load_peaks()
+    durs = measure_doc_pass(step, 2)          # per-layer document / suffix+merge times
+    doc_tfs = 4.0 * W.R * W.N * W.d * W.H / (durs["doc"] * 1e-3) / 1e12
     line = {"mode": "prefill", "metric": "prefill rows/s", "value": value, "unit": "rows/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
@@ -358,6 +360,8 @@ def mode_prefill(args, world, rank, local, dev):
                        "streams": W.P, "rows": W.R,
                        "l2": "per-layer document KV and question rows exceed L2"},
             "doc_tflops": tfs, "doc_frac_of_sustained_bf16": tfs / world / peaks["bf16_sustained"],
+            "per_layer_us": {"doc_pass": durs["doc"] * 1e3, "suffix_merge": durs["suffix"] * 1e3,
+                             "doc_pass_tflops": doc_tfs},
             "gpu_launches": step.kernels_per_step() * args.steps, "clocks": clocks}
     if rank == 0:
         print(json.dumps(line), flush=True)
