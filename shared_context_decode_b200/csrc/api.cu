@@ -125,9 +125,11 @@ long long wait_limit(const pp_options* opt) {
 
 // Shared body of decode and prefill attention.
 // causal: a document prefill; rows = doc_len document tokens, no stream ids.
+// read_once: a decode step (one row per stream), so each segment is read once.
 pp_status attend(const pp_kv_layer* L, int32_t doc_len, const uint16_t* q, const int16_t* q_sid,
                  const int32_t* q_pos, int32_t rows, float scale, uint16_t* o, float* lse, void* ws,
-                 size_t ws_bytes, const pp_options* opt, void* stream, bool causal = false) {
+                 size_t ws_bytes, const pp_options* opt, void* stream, bool causal = false,
+                 bool read_once = false) {
   pp_status s = check_layer(L);
   if (s != PP_OK) return s;
   if (rows < 0 || doc_len < 0) return PP_ERR_INVALID_ARG;
@@ -178,7 +180,7 @@ pp_status attend(const pp_kv_layer* L, int32_t doc_len, const uint16_t* q, const
       return s;
   } else if ((s = from_cuda(pp::launch_suffix_merge(*L, q, q_sid, q_pos, rows, scale, plan,
                                                     has_doc, part, o, lse, wait_limit(opt), sms,
-                                                    st))) != PP_OK) {
+                                                    read_once, st))) != PP_OK) {
     return s;
   }
   return from_cuda(mark(2));
@@ -273,7 +275,8 @@ PP_API pp_status pp_decode_attn(const pp_kv_layer* layer, int32_t doc_len, const
                          uint16_t* o, float* lse, void* ws, size_t ws_bytes, const pp_options* opt,
                          void* stream) {
   if (layer && P > layer->P_max) return PP_ERR_UNSUPPORTED;
-  return attend(layer, doc_len, q, q_sid, q_pos, P, scale, o, lse, ws, ws_bytes, opt, stream);
+  return attend(layer, doc_len, q, q_sid, q_pos, P, scale, o, lse, ws, ws_bytes, opt, stream,
+                false, true);
 }
 
 PP_API pp_status pp_prefill_attn(const pp_kv_layer* layer, int32_t doc_len, const uint16_t* q,

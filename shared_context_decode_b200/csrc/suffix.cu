@@ -70,6 +70,8 @@ struct SufParams {
   uint16_t* o;
   float* lse;
   long long wait_limit;
+  int read_once;   // 1: every segment is read by one row (decode), so its
+                   // copies are marked evict-first in L2
 };
 
 // Per-item record of the warp's table: stream id (0 when the row is not an
@@ -168,7 +170,10 @@ __global__ void __launch_bounds__(SufCfg<D>::WARPS * 32) suffix_merge(const SufP
   const bool doc_rows = p.q_sid == nullptr;
   const size_t seg_elems = (size_t)p.S_cap * D;
 
-  const uint64_t pol_first = l2_policy_evict_first();
+  // decode: each segment is read once, so its lines go first and the document
+  // partials the merge reads stay in L2; a question prefill re-reads a
+  // segment for every row of the question, so keep the default priority
+  const uint64_t pol = p.read_once ? l2_policy_evict_first() : l2_policy_evict_normal();
   uint32_t issued = 0, consumed = 0;
   bool ok = true;
   for (int64_t r0 = i_begin; ok && r0 < i_end; r0 += C::TBL) {
@@ -211,10 +216,8 @@ __global__ void __launch_bounds__(SufCfg<D>::WARPS * 32) suffix_merge(const SufP
         uint8_t* st = ring + stage * C::STAGE;
         fence_proxy_async();
         mbar_arrive_expect_tx(full + stage, 2u * nk * C::ROWB);
-        // evict-first: the rows are read once; the document partials the
-        // merge reads next stay in L2
-        bulk_load_hint(st, p.k_suf + seg, nk * C::ROWB, full + stage, pol_first);
-        bulk_load_hint(st + C::HALF, p.v_suf + seg, nk * C::ROWB, full + stage, pol_first);
+        bulk_load_hint(st, p.k_suf + seg, nk * C::ROWB, full + stage, pol);
+        bulk_load_hint(st + C::HALF, p.v_suf + seg, nk * C::ROWB, full + stage, pol);
       }
       pt0 += C::CK;
       return true;
@@ -454,7 +457,8 @@ __global__ void __launch_bounds__(SufCfg<D>::WARPS * 32) suffix_merge(const SufP
 cudaError_t launch_suffix_merge(const pp_kv_layer& L, const uint16_t* q, const int16_t* q_sid,
                                 const int32_t* q_pos, int rows, float scale, const SplitPlan& plan,
                                 bool has_doc, const Partials& part, uint16_t* o, float* lse,
-                                long long wait_limit, int num_sms, cudaStream_t st) {
+                                long long wait_limit, int num_sms, bool read_once,
+                                cudaStream_t st) {
   SufParams prm;
   prm.rows = rows;
   prm.H = L.H;
@@ -477,6 +481,7 @@ cudaError_t launch_suffix_merge(const pp_kv_layer& L, const uint16_t* q, const i
   prm.o = o;
   prm.lse = lse;
   prm.wait_limit = wait_limit;
+  prm.read_once = read_once ? 1 : 0;
   const int64_t items = (int64_t)rows * L.H;
   auto go = [&](auto kernel, int warps, int smem, std::atomic<uint64_t>& ready) -> cudaError_t {
     int dev = 0;
