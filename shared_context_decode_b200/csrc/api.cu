@@ -125,7 +125,9 @@ long long wait_limit(const pp_options* opt) {
 
 // Shared body of decode and prefill attention.
 // causal: a document prefill; rows = doc_len document tokens, no stream ids.
-// read_once: a decode step (one row per stream), so each segment is read once.
+// read_once: a decode step (one row per stream), so each segment is read once
+// and the per-row suffix kernel runs; otherwise rows come in question-sized
+// runs of one stream and the question-block kernel runs.
 pp_status attend(const pp_kv_layer* L, int32_t doc_len, const uint16_t* q, const int16_t* q_sid,
                  const int32_t* q_pos, int32_t rows, float scale, uint16_t* o, float* lse, void* ws,
                  size_t ws_bytes, const pp_options* opt, void* stream, bool causal = false,
@@ -178,9 +180,12 @@ pp_status attend(const pp_kv_layer* L, int32_t doc_len, const uint16_t* q, const
     if ((s = from_cuda(pp::launch_sibling_scan(*L, q, q_sid, q_pos, rows, scale, plan, has_doc,
                                                part, o, lse, st))) != PP_OK)
       return s;
-  } else if ((s = from_cuda(pp::launch_suffix_merge(*L, q, q_sid, q_pos, rows, scale, plan,
-                                                    has_doc, part, o, lse, wait_limit(opt), sms,
-                                                    read_once, st))) != PP_OK) {
+  } else if (read_once) {
+    if ((s = from_cuda(pp::launch_suffix_merge(*L, q, q_sid, q_pos, rows, scale, plan, has_doc,
+                                               part, o, lse, wait_limit(opt), sms, st))) != PP_OK)
+      return s;
+  } else if ((s = from_cuda(pp::launch_suffix_block(*L, q, q_sid, q_pos, rows, scale, plan,
+                                                    has_doc, part, o, lse, sms, st))) != PP_OK) {
     return s;
   }
   return from_cuda(mark(2));

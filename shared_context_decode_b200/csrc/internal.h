@@ -37,12 +37,18 @@ cudaError_t launch_sibling_scan(const pp_kv_layer& L, const uint16_t* q, const i
                                 const int32_t* q_pos, int rows, float scale, const SplitPlan& plan,
                                 bool has_doc, const Partials& part, uint16_t* o, float* lse,
                                 cudaStream_t st);
-// Suffix pass with the log-sum-exp merge in its epilogue; writes o and lse.
+// Suffix pass of a decode step (one warp per row and head) with the
+// log-sum-exp merge in its epilogue; writes o and lse.
 cudaError_t launch_suffix_merge(const pp_kv_layer& L, const uint16_t* q, const int16_t* q_sid,
                                 const int32_t* q_pos, int rows, float scale, const SplitPlan& plan,
                                 bool has_doc, const Partials& part, uint16_t* o, float* lse,
-                                long long wait_limit, int num_sms, bool read_once,
-                                cudaStream_t st);
+                                long long wait_limit, int num_sms, cudaStream_t st);
+// Suffix pass of a prefill call (one warp per 16 rows and head, warp-level
+// mma), merge first; q_sid = nullptr for document rows.  Writes o and lse.
+cudaError_t launch_suffix_block(const pp_kv_layer& L, const uint16_t* q, const int16_t* q_sid,
+                                const int32_t* q_pos, int rows, float scale, const SplitPlan& plan,
+                                bool has_doc, const Partials& part, uint16_t* o, float* lse,
+                                int num_sms, cudaStream_t st);
 cudaError_t launch_visibility(const pp_kv_layer& L, int doc_len, const int16_t* q_sid,
                               const int32_t* q_pos, int nq, int32_t* count_out, uint8_t* mask_out,
                               cudaStream_t st);

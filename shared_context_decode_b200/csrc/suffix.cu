@@ -3,8 +3,9 @@
 // Each query row attends, besides the document, to the slots of its own
 // stream segment that the stream mask admits ("Read Once, Answer Many"
 // project page, section "How it works", item 1: same stream id and not later
-// than the query).  The decode step (one row per stream) and the question
-// prefill (rows causal within their question) run the same kernel.
+// than the query).  This kernel serves decode steps (one row per stream, so
+// every segment is read by one row); prefill calls, whose rows share their
+// question's segment, run the question-block kernel of suffix_block.cu.
 //
 // Work item = (query row, head).  Each warp owns a contiguous, balanced block
 // of items and a ring of NS shared-memory stages; lane 0 fills them with 1-D
@@ -70,8 +71,6 @@ struct SufParams {
   uint16_t* o;
   float* lse;
   long long wait_limit;
-  int read_once;   // 1: every segment is read by one row (decode), so its
-                   // copies are marked evict-first in L2
 };
 
 // Per-item record of the warp's table: stream id (0 when the row is not an
@@ -170,10 +169,9 @@ __global__ void __launch_bounds__(SufCfg<D>::WARPS * 32) suffix_merge(const SufP
   const bool doc_rows = p.q_sid == nullptr;
   const size_t seg_elems = (size_t)p.S_cap * D;
 
-  // decode: each segment is read once, so its lines go first and the document
-  // partials the merge reads stay in L2; a question prefill re-reads a
-  // segment for every row of the question, so keep the default priority
-  const uint64_t pol = p.read_once ? l2_policy_evict_first() : l2_policy_evict_normal();
+  // each segment is read once, so its lines go first and the document
+  // partials the merge reads stay in L2
+  const uint64_t pol = l2_policy_evict_first();
   uint32_t issued = 0, consumed = 0;
   bool ok = true;
   for (int64_t r0 = i_begin; ok && r0 < i_end; r0 += C::TBL) {
@@ -457,7 +455,7 @@ __global__ void __launch_bounds__(SufCfg<D>::WARPS * 32) suffix_merge(const SufP
 cudaError_t launch_suffix_merge(const pp_kv_layer& L, const uint16_t* q, const int16_t* q_sid,
                                 const int32_t* q_pos, int rows, float scale, const SplitPlan& plan,
                                 bool has_doc, const Partials& part, uint16_t* o, float* lse,
-                                long long wait_limit, int num_sms, bool read_once,
+                                long long wait_limit, int num_sms,
                                 cudaStream_t st) {
   SufParams prm;
   prm.rows = rows;
@@ -481,7 +479,6 @@ cudaError_t launch_suffix_merge(const pp_kv_layer& L, const uint16_t* q, const i
   prm.o = o;
   prm.lse = lse;
   prm.wait_limit = wait_limit;
-  prm.read_once = read_once ? 1 : 0;
   const int64_t items = (int64_t)rows * L.H;
   auto go = [&](auto kernel, int warps, int smem, std::atomic<uint64_t>& ready) -> cudaError_t {
     int dev = 0;
