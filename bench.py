@@ -188,20 +188,30 @@ class DecodeStep:
         torch.cuda.synchronize()
         self.len0 = self.len_all.clone()
         self.opts = None   # per-layer pp_options of the captured step (None = default)
+        # one pp_decode_step per layer (the append inside the document pass);
+        # False: pp_kv_append then pp_decode_attn, for comparison
+        self.fused = True
         self.ws = pp.workspace(pp.decode_workspace_bytes(W.P, W.H, W.d, W.N), device)
         self.graph = None
+
+    def layer_call(self, l, opt):
+        """Append layer l's decode tokens and attend."""
+        pp, x = self.pp, self.inp[l]
+        if self.fused:
+            pp.decode_step(self.cache[l], self.W.N, x["k"], x["v"], x["q"], x["sid"], x["pos"],
+                           self.W.scale, o=x["o"], ws=self.ws, opt=opt)
+        else:
+            pp.kv_append(self.cache[l], x["k"], x["v"], x["sid"], x["pos"])
+            pp.decode_attn(self.cache[l], self.W.N, x["q"], x["sid"], x["pos"], self.W.scale,
+                           o=x["o"], ws=self.ws, opt=opt)
 
     def run_eager(self, opts=None):
         """One decode step, launched eagerly (also the body that is captured);
         opts: per-layer pp_options or None."""
-        pp = self.pp
         opts = opts if opts is not None else self.opts
         self.len_all.copy_(self.len0)
         for l in range(self.layers):
-            x = self.inp[l]
-            pp.kv_append(self.cache[l], x["k"], x["v"], x["sid"], x["pos"])
-            pp.decode_attn(self.cache[l], self.W.N, x["q"], x["sid"], x["pos"], self.W.scale,
-                           o=x["o"], ws=self.ws, opt=None if opts is None else opts[l])
+            self.layer_call(l, None if opts is None else opts[l])
 
     def capture(self):
         self.run_eager()           # warm: per-device setup happens outside the capture
@@ -246,10 +256,7 @@ class DecodeStep:
                 for l in range(self.layers):
                     x = self.inp[l]
                     comp.wait_event(ev_in[l])
-                    pp.kv_append(self.cache[l], x["k"], x["v"], x["sid"], x["pos"])
-                    pp.decode_attn(self.cache[l], self.W.N, x["q"], x["sid"], x["pos"],
-                                   self.W.scale, o=x["o"], ws=self.ws,
-                                   opt=None if self.opts is None else self.opts[l])
+                    self.layer_call(l, None if self.opts is None else self.opts[l])
                     e = torch.cuda.Event()
                     e.record(comp)
                     cout.wait_event(e)
@@ -262,8 +269,15 @@ class DecodeStep:
         self.graph_e2e = g
 
     def kernels_per_step(self) -> int:
-        # per layer: append (rows + lengths) 2, document pass 1, suffix pass + merge 1
-        return self.layers * 4
+        # per layer: the document pass (carrying the append) and the suffix
+        # pass + merge; the append's own two kernels when it runs separately
+        # (unfused, or beside the ablation and sibling-scan modes)
+        n = 0
+        for l in range(self.layers):
+            o = None if self.opts is None else self.opts[l]
+            other = o is not None and (o.ablation_doc_per_stream or o.sibling_scan)
+            n += 4 if (not self.fused or other or self.W.N == 0) else 2
+        return n
 
     def check_status(self):
         for kv in self.cache:
@@ -710,6 +724,9 @@ def main():
                     help="CPU-baseline sample budget (0 = skip)")
     ap.add_argument("--ref-seconds", type=float, default=10.0)
     ap.add_argument("--roofline-reps", type=int, default=3)
+    ap.add_argument("--separate-append", action="store_true",
+                    help="decode: pp_kv_append + pp_decode_attn per layer instead of "
+                         "pp_decode_step (append inside the document pass), for comparison")
     ap.add_argument("--mode", default="decode",
                     choices=["decode", "prefill", "ablation", "siblingscan", "sweep", "docprefill"],
                     help="decode: the headline step (default); others: secondary measurements")
@@ -741,6 +758,7 @@ def main():
     from shared_context_decode_b200 import workloads as wl
     nl = args.layers or wl.CONFIGS[args.workload]["layers"]
     step = DecodeStep(args.workload, nl, dev)
+    step.fused = not args.separate_append
     W = step.W
     step.capture()
 
@@ -830,6 +848,8 @@ def main():
                        "suffix_tokens": W.suffix_tokens(),
                        "l2": "inputs larger than L2 (8.6 GB of document KV per step)"
                              if nl == 32 else "per-layer document KV exceeds L2",
+                       "append": "inside the document pass (pp_decode_step)" if step.fused
+                                 else "separate kernels (pp_kv_append)",
                        "parallelism": f"replicas x{world}"},
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},

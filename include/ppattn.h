@@ -198,6 +198,29 @@ pp_status pp_decode_attn(const pp_kv_layer *layer, int32_t doc_len, const uint16
                          const pp_options *opt, void *stream);
 
 /*
+ * One decode step of a layer in one call: append each row's new token, then
+ * attend ("How it works": a decode step appends one token per stream, then
+ * every stream's query reads the shared document once and its own segment).
+ *   k, v   bf16 [P][H][d]   the new tokens' keys and values; row i is
+ *                           appended to stream q_sid[i] at position q_pos[i]
+ *   the other arguments and the workspace size are those of pp_decode_attn.
+ * The result equals pp_kv_append(k, v, q_sid, q_pos, P) followed by
+ * pp_decode_attn(...) -- the same slots, tags, lengths, device flags and
+ * outputs -- except that rows of stream 0 are not written to the document
+ * (a decode step has no document rows; they are flagged PP_DEV_BAD_STREAM as
+ * in pp_decode_attn).  With a document and at most 4096 rows the append runs
+ * inside the document pass launch, on a warp that is otherwise idle, and the
+ * suffix pass stores the advanced lengths: two kernel launches per layer
+ * instead of four.  Otherwise (doc_len 0, more rows, or the ablation and
+ * sibling-scan options) the append kernels run first.  k and v: 16-byte
+ * aligned.  Asynchronous, capture-safe.
+ */
+pp_status pp_decode_step(const pp_kv_layer *layer, int32_t doc_len, const uint16_t *k,
+                         const uint16_t *v, const uint16_t *q, const int16_t *q_sid,
+                         const int32_t *q_pos, int32_t P, float scale, uint16_t *o, float *lse,
+                         void *ws, size_t ws_bytes, const pp_options *opt, void *stream);
+
+/*
  * pp_decode_attn for callers that cannot allocate device memory.  The pages
  * have no counterpart: this is a library convenience.
  *

@@ -97,18 +97,25 @@ SplitPlan plan_for(int rows, int H, int doc_len, const pp_options* opt, bool cau
 }
 
 struct WsLayout {
-  size_t doc_o, doc_ml, total;
+  size_t doc_o, doc_ml, row_len, total;
 };
 
-// Only the document pass leaves partial results in the workspace.
+// The document pass leaves its partial results in the workspace and, in a
+// decode step whose append it carries, each row's stream length (one int per
+// row; not needed by the causal document prefill).
 WsLayout ws_layout(const SplitPlan& p, int d) {
   WsLayout w;
   const size_t slots = (size_t)p.units * p.max_chunks * pp::kGroupRows;
   w.doc_o = 0;
   w.doc_ml = w.doc_o + up(slots * d * sizeof(float));
-  w.total = w.doc_ml + up(slots * 2 * sizeof(float));
+  w.row_len = w.doc_ml + up(slots * 2 * sizeof(float));
+  w.total = w.row_len + (slots && !p.causal ? up((size_t)p.G * pp::kGroupRows * sizeof(int32_t)) : 0);
   return w;
 }
+
+// Largest decode step whose append runs inside the document pass: every
+// appended row counts its stream's rows over the whole call.
+constexpr int kFusedAppendMaxRows = 4096;
 
 Partials carve(void* ws, const WsLayout& w) {
   uint8_t* b = static_cast<uint8_t*>(ws);
@@ -125,13 +132,18 @@ long long wait_limit(const pp_options* opt) {
 
 // Shared body of decode and prefill attention.
 // causal: a document prefill; rows = doc_len document tokens, no stream ids.
+// app_k, app_v: a decode step's new keys and values (one row per query row,
+// the rows' own stream ids and positions), appended before the attention:
+// inside the document pass launch when there is one, else by the append
+// kernels; nullptr: nothing to append.
 // read_once: a decode step (one row per stream), so each segment is read once
 // and the per-row suffix kernel runs; otherwise rows come in question-sized
 // runs of one stream and the question-block kernel runs.
 pp_status attend(const pp_kv_layer* L, int32_t doc_len, const uint16_t* q, const int16_t* q_sid,
                  const int32_t* q_pos, int32_t rows, float scale, uint16_t* o, float* lse, void* ws,
                  size_t ws_bytes, const pp_options* opt, void* stream, bool causal = false,
-                 bool read_once = false) {
+                 bool read_once = false, const uint16_t* app_k = nullptr,
+                 const uint16_t* app_v = nullptr) {
   pp_status s = check_layer(L);
   if (s != PP_OK) return s;
   if (rows < 0 || doc_len < 0) return PP_ERR_INVALID_ARG;
@@ -165,6 +177,17 @@ pp_status attend(const pp_kv_layer* L, int32_t doc_len, const uint16_t* q, const
                ? cudaEventRecordWithFlags(ev[i], st, cudaEventRecordExternal)
                : cudaEventRecord(ev[i], st);
   };
+  const bool other_doc = opt && (opt->ablation_doc_per_stream || opt->sibling_scan);
+  pp::AppendJob app{};
+  if (app_k) {
+    if (has_doc && !other_doc && rows <= kFusedAppendMaxRows) {
+      app = {app_k, app_v, q_sid, q_pos, rows,
+             reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + w.row_len)};
+    } else if ((s = from_cuda(pp::launch_kv_append(*L, app_k, app_v, q_sid, q_pos, rows, st,
+                                                   true))) != PP_OK) {
+      return s;
+    }
+  }
   if (mark(0) != cudaSuccess) return PP_ERR_CUDA;
   if (has_doc) {
     cudaError_t e;
@@ -172,7 +195,7 @@ pp_status attend(const pp_kv_layer* L, int32_t doc_len, const uint16_t* q, const
       e = pp::launch_doc_per_stream(*L, doc_len, q, rows, scale, plan.max_chunks, part, st);
     else
       e = pp::launch_doc_pass_tc(*L, doc_len, q, rows, scale, plan, part, wait_limit(opt),
-                                 opt ? opt->debug_inject_timeout : 0, st);
+                                 opt ? opt->debug_inject_timeout : 0, app, st);
     if (e != cudaSuccess) return PP_ERR_CUDA;
   }
   if (mark(1) != cudaSuccess) return PP_ERR_CUDA;
@@ -182,7 +205,8 @@ pp_status attend(const pp_kv_layer* L, int32_t doc_len, const uint16_t* q, const
       return s;
   } else if (read_once) {
     if ((s = from_cuda(pp::launch_suffix_merge(*L, q, q_sid, q_pos, rows, scale, plan, has_doc,
-                                               part, o, lse, wait_limit(opt), sms, st))) != PP_OK)
+                                               part, o, lse, wait_limit(opt), sms,
+                                               app.n ? app.row_len : nullptr, st))) != PP_OK)
       return s;
   } else if ((s = from_cuda(pp::launch_suffix_block(*L, q, q_sid, q_pos, rows, scale, plan,
                                                     has_doc, part, o, lse, sms, st))) != PP_OK) {
@@ -282,6 +306,17 @@ PP_API pp_status pp_decode_attn(const pp_kv_layer* layer, int32_t doc_len, const
   if (layer && P > layer->P_max) return PP_ERR_UNSUPPORTED;
   return attend(layer, doc_len, q, q_sid, q_pos, P, scale, o, lse, ws, ws_bytes, opt, stream,
                 false, true);
+}
+
+PP_API pp_status pp_decode_step(const pp_kv_layer* layer, int32_t doc_len, const uint16_t* k,
+                                const uint16_t* v, const uint16_t* q, const int16_t* q_sid,
+                                const int32_t* q_pos, int32_t P, float scale, uint16_t* o,
+                                float* lse, void* ws, size_t ws_bytes, const pp_options* opt,
+                                void* stream) {
+  if (layer && P > layer->P_max) return PP_ERR_UNSUPPORTED;
+  if (P > 0 && (!k || !v || !aligned(k, 16) || !aligned(v, 16))) return PP_ERR_INVALID_ARG;
+  return attend(layer, doc_len, q, q_sid, q_pos, P, scale, o, lse, ws, ws_bytes, opt, stream,
+                false, true, k, v);
 }
 
 PP_API pp_status pp_prefill_attn(const pp_kv_layer* layer, int32_t doc_len, const uint16_t* q,

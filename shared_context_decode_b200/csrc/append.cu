@@ -15,10 +15,11 @@ namespace pp {
 __global__ void __launch_bounds__(128) kv_append_rows(pp_kv_layer L, const uint4* __restrict__ k,
                                                       const uint4* __restrict__ v,
                                                       const int16_t* __restrict__ sid,
-                                                      const int32_t* __restrict__ pos, int n) {
+                                                      const int32_t* __restrict__ pos, int n,
+                                                      int streams_only) {
   const int i = blockIdx.x;
   const int s = sid[i];
-  if (s < 0) return;
+  if (s < 0 || (s == 0 && streams_only)) return;
   const int vec_per_head = L.d / 8;  // 16-byte vectors of 8 bf16
   const int vec_per_row = L.H * vec_per_head;
   const uint4* krow = k + (int64_t)i * vec_per_row;
@@ -114,9 +115,11 @@ cudaError_t launch_kv_reset_streams(const pp_kv_layer& L, const int16_t* sid, in
 }
 
 cudaError_t launch_kv_append(const pp_kv_layer& L, const uint16_t* k, const uint16_t* v,
-                             const int16_t* sid, const int32_t* pos, int n, cudaStream_t st) {
+                             const int16_t* sid, const int32_t* pos, int n, cudaStream_t st,
+                             bool streams_only) {
   kv_append_rows<<<n, 128, 0, st>>>(L, reinterpret_cast<const uint4*>(k),
-                                    reinterpret_cast<const uint4*>(v), sid, pos, n);
+                                    reinterpret_cast<const uint4*>(v), sid, pos, n,
+                                    streams_only ? 1 : 0);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int blocks = (n + 255) / 256 < 148 ? (n + 255) / 256 : 148;

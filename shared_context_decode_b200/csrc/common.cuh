@@ -197,6 +197,17 @@ struct Partials {
   float* doc_ml;    // [units*max_chunks][kGroupRows][2]  (max, sum), log2 domain
 };
 
+// A decode step's append, carried out by one otherwise idle warp of each CTA
+// of the document pass (append_warp.cuh).  n = 0: nothing to append.
+struct AppendJob {
+  const uint16_t* k;   // [n, H, d] bf16, the decode tokens' keys
+  const uint16_t* v;   // [n, H, d] bf16
+  const int16_t* sid;  // [n] stream ids (the query rows' own)
+  const int32_t* pos;  // [n] positions
+  int n;
+  int32_t* row_len;    // [n] out: length of row i's stream after the call
+};
+
 // ---------------------------------------------------------------------------
 // PTX wrappers: shared-memory mbarriers, TMA, tcgen05.
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {

@@ -39,6 +39,7 @@
 #include <atomic>
 #include <mutex>
 
+#include "append_warp.cuh"
 #include "common.cuh"
 #include "internal.h"
 
@@ -63,6 +64,8 @@ struct DocTcParams {
   int32_t* status;
   long long wait_limit;
   int inject_timeout;
+  AppendJob app;  // a decode step's append, done by warp 2 (n = 0: none)
+  pp_kv_layer L;
 };
 
 template <int D>
@@ -403,7 +406,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else if (warp == 2) {
+    // ------------------------------- TMEM owner; idle until the teardown ----
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLow));
+    if (p.app.n > 0) append_pairs_warp<D>(p.app, p.L, blockIdx.x, gridDim.x, lane);
   } else {
     // ---------------------------------------------------------- softmax ----
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsHigh));
@@ -633,7 +638,7 @@ namespace {
 template <int D>
 cudaError_t launch_impl(const pp_kv_layer& L, int doc_len, const uint16_t* q, int rows, float scale,
                         const SplitPlan& plan, const Partials& part, long long wait_limit,
-                        int inject, cudaStream_t st) {
+                        int inject, const AppendJob& app, cudaStream_t st) {
   using C = DocCfg<D>;
   CUtensorMap mQ, mK, mV;
   if (!make_tmap_bf16_3d(&mQ, q, D, L.H, rows, (uint64_t)D * 2, (uint64_t)L.H * D * 2, 64, 1, 128) ||
@@ -672,6 +677,8 @@ cudaError_t launch_impl(const pp_kv_layer& L, int doc_len, const uint16_t* q, in
   prm.status = L.status;
   prm.wait_limit = wait_limit;
   prm.inject_timeout = inject;
+  prm.app = app;
+  prm.L = L;
   doc_pass_tc<D><<<plan.C * prm.pair, kThreads, C::SMEM, st>>>(mQ, mK, mV, prm);
   return cudaGetLastError();
 }
@@ -680,10 +687,13 @@ cudaError_t launch_impl(const pp_kv_layer& L, int doc_len, const uint16_t* q, in
 
 cudaError_t launch_doc_pass_tc(const pp_kv_layer& L, int doc_len, const uint16_t* q, int rows,
                                float scale, const SplitPlan& plan, const Partials& part,
-                               long long wait_limit, int inject_timeout, cudaStream_t st) {
+                               long long wait_limit, int inject_timeout, const AppendJob& app,
+                               cudaStream_t st) {
   if (L.d == 128)
-    return launch_impl<128>(L, doc_len, q, rows, scale, plan, part, wait_limit, inject_timeout, st);
-  return launch_impl<64>(L, doc_len, q, rows, scale, plan, part, wait_limit, inject_timeout, st);
+    return launch_impl<128>(L, doc_len, q, rows, scale, plan, part, wait_limit, inject_timeout,
+                            app, st);
+  return launch_impl<64>(L, doc_len, q, rows, scale, plan, part, wait_limit, inject_timeout, app,
+                         st);
 }
 
 }  // namespace pp

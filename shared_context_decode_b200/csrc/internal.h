@@ -18,16 +18,23 @@ bool make_tmap_bf16_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d
                        uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t b0, uint32_t b1,
                        uint32_t b2);
 
+struct AppendJob;
+
+// streams_only: rows of stream 0 are skipped instead of written to the
+// document block (a decode step carries no document rows).
 cudaError_t launch_kv_append(const pp_kv_layer& L, const uint16_t* k, const uint16_t* v,
-                             const int16_t* sid, const int32_t* pos, int n, cudaStream_t st);
+                             const int16_t* sid, const int32_t* pos, int n, cudaStream_t st,
+                             bool streams_only = false);
 cudaError_t launch_kv_reset(const pp_kv_layer& L, cudaStream_t st);
 cudaError_t launch_kv_reset_streams(const pp_kv_layer& L, const int16_t* sid, int n,
                                     cudaStream_t st);
 
-// Document pass on the tensor cores; tensor maps are built inside.
+// Document pass on the tensor cores; tensor maps are built inside.  app: a
+// decode step's append, done inside the launch (app.n = 0: none).
 cudaError_t launch_doc_pass_tc(const pp_kv_layer& L, int doc_len, const uint16_t* q, int rows,
                                float scale, const SplitPlan& plan, const Partials& part,
-                               long long wait_limit, int inject_timeout, cudaStream_t st);
+                               long long wait_limit, int inject_timeout, const AppendJob& app,
+                               cudaStream_t st);
 cudaError_t launch_doc_per_stream(const pp_kv_layer& L, int doc_len, const uint16_t* q, int rows,
                                   float scale, int max_chunks, const Partials& part,
                                   cudaStream_t st);
@@ -38,11 +45,14 @@ cudaError_t launch_sibling_scan(const pp_kv_layer& L, const uint16_t* q, const i
                                 bool has_doc, const Partials& part, uint16_t* o, float* lse,
                                 cudaStream_t st);
 // Suffix pass of a decode step (one warp per row and head) with the
-// log-sum-exp merge in its epilogue; writes o and lse.
+// log-sum-exp merge in its epilogue; writes o and lse.  row_len: the stream
+// lengths left by an append inside the document pass, per row (stored into
+// len by this kernel); nullptr: read len.
 cudaError_t launch_suffix_merge(const pp_kv_layer& L, const uint16_t* q, const int16_t* q_sid,
                                 const int32_t* q_pos, int rows, float scale, const SplitPlan& plan,
                                 bool has_doc, const Partials& part, uint16_t* o, float* lse,
-                                long long wait_limit, int num_sms, cudaStream_t st);
+                                long long wait_limit, int num_sms, const int32_t* row_len,
+                                cudaStream_t st);
 // Suffix pass of a prefill call (one warp per 16 rows and head, warp-level
 // mma), merge first; q_sid = nullptr for document rows.  Writes o and lse.
 cudaError_t launch_suffix_block(const pp_kv_layer& L, const uint16_t* q, const int16_t* q_sid,

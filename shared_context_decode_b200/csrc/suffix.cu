@@ -61,7 +61,10 @@ struct SufParams {
   const uint16_t* v_suf;
   const int16_t* sid;
   const int32_t* pos;
-  const int32_t* len;
+  int32_t* len;
+  // decode step whose append ran inside the document pass: row r's stream
+  // length is row_len[r], and this kernel stores it into len (nullptr: read len)
+  const int32_t* row_len;
   int32_t* status;
   float sl2;
   SplitPlan plan;
@@ -192,7 +195,14 @@ __global__ void __launch_bounds__(SufCfg<D>::WARPS * 32) suffix_merge(const SufP
     for (int k = lane; k < cnt; k += 32) {
       const int s = tbl[k].s;
       if (s) {
-        const int n = p.len[s - 1];
+        int n;
+        if (p.row_len) {
+          const int64_t item = r0 + k;
+          n = p.row_len[item % p.rows];
+          if (item < p.rows) p.len[s - 1] = n;   // head 0's items store the advanced length
+        } else {
+          n = p.len[s - 1];
+        }
         tbl[k].n = n < p.S_cap ? n : p.S_cap;
       }
     }
@@ -455,7 +465,7 @@ __global__ void __launch_bounds__(SufCfg<D>::WARPS * 32) suffix_merge(const SufP
 cudaError_t launch_suffix_merge(const pp_kv_layer& L, const uint16_t* q, const int16_t* q_sid,
                                 const int32_t* q_pos, int rows, float scale, const SplitPlan& plan,
                                 bool has_doc, const Partials& part, uint16_t* o, float* lse,
-                                long long wait_limit, int num_sms,
+                                long long wait_limit, int num_sms, const int32_t* row_len,
                                 cudaStream_t st) {
   SufParams prm;
   prm.rows = rows;
@@ -470,6 +480,7 @@ cudaError_t launch_suffix_merge(const pp_kv_layer& L, const uint16_t* q, const i
   prm.sid = L.sid;
   prm.pos = L.pos;
   prm.len = L.len;
+  prm.row_len = row_len;
   prm.status = L.status;
   prm.sl2 = scale * kLog2e;
   prm.plan = plan;

@@ -82,6 +82,8 @@ _dec_ws = _sig("pp_decode_workspace_bytes", _sz, _i32, _i32, _i32, _i32, _OP)
 _pre_ws = _sig("pp_prefill_workspace_bytes", _sz, _i32, _i32, _i32, _i32, _OP)
 _decode = _sig("pp_decode_attn", _i32, _LP, _i32, _vp, _vp, _vp, _i32, ctypes.c_float, _vp, _vp,
                _vp, _sz, _OP, _vp)
+_decode_step = _sig("pp_decode_step", _i32, _LP, _i32, _vp, _vp, _vp, _vp, _vp, _i32,
+                    ctypes.c_float, _vp, _vp, _vp, _sz, _OP, _vp)
 _decode_noalloc = _sig("pp_decode_attn_noalloc", _i32, _LP, _i32, _vp, _vp, _vp, _i32,
                       ctypes.c_float, _vp, _vp, _OP, _vp)
 _prefill = _sig("pp_prefill_attn", _i32, _LP, _i32, _vp, _vp, _vp, _i32, ctypes.c_float, _vp,
@@ -103,7 +105,7 @@ EXPORTED = ("pp_status_str", "pp_abi_version", "pp_kv_reset", "pp_kv_append",
             "pp_prefill_attn", "pp_debug_visibility", "pp_get_device_status",
             "pp_debug_split_plan", "pp_debug_exp2", "pp_decode_attn_noalloc",
             "pp_doc_prefill_workspace_bytes", "pp_doc_prefill_attn", "pp_debug_split_plan_causal",
-            "pp_kv_reset_streams")
+            "pp_kv_reset_streams", "pp_decode_step")
 
 # Size of the scratch array built into the library for pp_decode_attn_noalloc.
 NOALLOC_SCRATCH_BYTES = 32 << 20
@@ -296,6 +298,27 @@ def decode_attn(layer: KVLayer, doc_len: int, q: torch.Tensor, q_sid: torch.Tens
     """Decode-step attention of P query rows; returns o [P, H, d] bf16."""
     return _attn(_decode, "pp_decode_attn", layer, doc_len, q, q_sid, q_pos, scale, o, lse, ws,
                  opt, decode_workspace_bytes)
+
+
+def decode_step(layer: KVLayer, doc_len: int, k: torch.Tensor, v: torch.Tensor, q: torch.Tensor,
+                q_sid: torch.Tensor, q_pos: torch.Tensor, scale: float,
+                o: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                ws: Optional[torch.Tensor] = None, opt: Optional[Options] = None) -> torch.Tensor:
+    """One decode step of a layer: append row i's k/v to stream q_sid[i] at
+    q_pos[i], then attend; returns o [P, H, d] bf16."""
+    dev = layer.device
+    rows = q_sid.shape[0]
+    for t, nm in ((k, "k"), (v, "v")):
+        _want(t, torch.bfloat16, nm, dev)
+        if t.shape != (rows, layer.H, layer.d):
+            raise ValueError(f"pp_decode_step: {nm} must be [rows, H, d]")
+
+    def fn(ref, doc_len_, qp, sp, pp_, n, sc, op, lp, wp, wn, optp, st):
+        return _decode_step(ref, doc_len_, _ptr(k), _ptr(v), qp, sp, pp_, n, sc, op, lp, wp, wn,
+                            optp, st)
+
+    return _attn(fn, "pp_decode_step", layer, doc_len, q, q_sid, q_pos, scale, o, lse, ws, opt,
+                 decode_workspace_bytes)
 
 
 def decode_attn_noalloc(layer: KVLayer, doc_len: int, q: torch.Tensor, q_sid: torch.Tensor,

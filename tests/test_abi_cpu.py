@@ -87,6 +87,20 @@ def test_host_validation_codes(pp):
     # prefill
     assert pp._prefill(ctypes.byref(L), 2000, 0x90000, 0xA0000, 0xB0000, 5, 0.1, 0xC0000, None,
                        0xD0000, 1 << 30, None, None) == pp.PP_ERR_CAPACITY
+    # fused decode step: the attention checks, plus k and v
+    def step(k=0xE0000, v=0xF0000, **kw):
+        a = dict(doc_len=10, P=4, q=0x90000, ws=1 << 30)
+        a.update(kw)
+        return pp._decode_step(ctypes.byref(a.pop("L", L)), a["doc_len"], k, v, a["q"], 0xA0000,
+                               0xB0000, a["P"], 0.1, 0xC0000, None, 0xD0000, a["ws"], None, None)
+    assert step(P=9) == pp.PP_ERR_UNSUPPORTED                          # P > P_max
+    assert step(k=0) == pp.PP_ERR_INVALID_ARG
+    assert step(v=0xF0008) == pp.PP_ERR_INVALID_ARG                    # misaligned v
+    assert step(q=0x90004) == pp.PP_ERR_INVALID_ARG
+    assert step(doc_len=1025) == pp.PP_ERR_CAPACITY
+    assert step(ws=16) == pp.PP_ERR_CAPACITY
+    assert step(P=0) == pp.PP_OK
+    assert step(L=fake_layer(pp, d=96)) == pp.PP_ERR_UNSUPPORTED
     # visibility
     assert pp._visibility(ctypes.byref(L), 5, 0x1000, 0x2000, -1, 0x3000, None, None) == \
         pp.PP_ERR_INVALID_ARG
@@ -97,7 +111,10 @@ def test_workspace_sizes_with_explicit_split(pp):
     ws = pp.decode_workspace_bytes(256, 32, 128, 16384, opt)
     plan = pp.split_plan(256, 32, 16384, 148)
     slots = plan["units"] * plan["max_chunks"] * 256
-    expect = slots * 128 * 4 + slots * 2 * 4       # document partials (O; max and sum)
+    groups = plan["units"] // 32
+    # document partials (O; max and sum), then one stream length per row
+    # (rounded up to whole row groups) for a step whose append the pass carries
+    expect = slots * 128 * 4 + slots * 2 * 4 + groups * 256 * 4
     assert ws == expect
     assert pp.decode_workspace_bytes(4, 4, 96, 10, opt) == 0
     # no document: nothing to carry between kernels
