@@ -414,6 +414,42 @@ def mode_ablation(args, world, rank, local, dev, sibling=False):
     del step.graph
 
 
+def mode_longanswer(args, world, rank, local, dev):
+    """Decode step with long answers (1024 cached answer tokens per stream):
+    the suffix pass dominates.  Timed with the automatic slicing of the
+    suffix work (the value) and with each slicing forced."""
+    from shared_context_decode_b200 import workloads as wl
+    name = "doc8k_p128_a1k"
+    nl = args.layers or wl.CONFIGS[name]["layers"]
+    step = DecodeStep(name, nl, dev)
+    pp, W = step.pp, step.W
+    runs = {}
+    for mode, sl in (("automatic", 0), ("equal_items", 1), ("balanced", 2)):
+        step.opts = [pp.Options(suffix_slices=sl) for _ in range(nl)]
+        step.capture()
+        ms, clocks = timed_replays(step, args.steps, args.warmup, world, local)
+        step.check_status()
+        per = measure_doc_pass(step, args.roofline_reps)
+        runs[mode] = {"ms_per_step": ms, "doc_us": per["doc"], "suffix_merge_us": per["suffix"],
+                      "clocks": clocks}
+        del step.graph
+    ms = runs["automatic"]["ms_per_step"]
+    value, ms = aggregate(W.P, ms, world, dev)
+    suf_bytes = W.suffix_tokens() * W.H * W.d * 2 * 2 + W.P * W.H * W.d * 2 * 2
+    line = {"mode": "longanswer", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": name, "layers": nl, "H": W.H, "d": W.d, "doc_tokens": W.N,
+                       "streams": W.P, "suffix_tokens": W.suffix_tokens()},
+            "suffix_bytes_per_layer": suf_bytes,
+            "suffix_hbm_gbs": {k: suf_bytes / (v["suffix_merge_us"] * 1e3) for k, v in runs.items()},
+            "runs": runs, "gpu_launches": step.kernels_per_step() * args.steps * 3,
+            "clocks": runs["automatic"]["clocks"]}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def mode_docprefill(args, world, rank, local, dev):
     """Document prefill: per layer, causal attention of the document's own
     tokens with the document K/V already cached (written once, outside the
@@ -581,7 +617,7 @@ def doc_pass_algorithmic(W):
 
 
 DOC_PROFILE = os.path.join(ROOT, "profiles", "doc_pass_tc_doc16k_p256.md")
-DOC_SOURCES = ("doc_tc.cu", "common.cuh")
+DOC_SOURCES = ("doc_tc.cu", "append_warp.cuh", "common.cuh")
 
 
 def kernel_source_hash(files=DOC_SOURCES) -> str:
@@ -633,6 +669,10 @@ def measure_doc_pass(step: DecodeStep, reps: int):
     opts = []
     for l in range(step.layers):
         o = pp.Options()
+        if step.opts is not None:   # same kernels as the timed step, plus the events
+            for f, _ in pp.Options._fields_:
+                if f != "events":
+                    setattr(o, f, getattr(step.opts[l], f))
         o.set_events(evs[l])
         opts.append(o)
     g = torch.cuda.CUDAGraph()
@@ -728,7 +768,8 @@ def main():
                     help="decode: pp_kv_append + pp_decode_attn per layer instead of "
                          "pp_decode_step (append inside the document pass), for comparison")
     ap.add_argument("--mode", default="decode",
-                    choices=["decode", "prefill", "ablation", "siblingscan", "sweep", "docprefill"],
+                    choices=["decode", "prefill", "ablation", "siblingscan", "sweep", "docprefill",
+                             "longanswer"],
                     help="decode: the headline step (default); others: secondary measurements")
     args = ap.parse_args()
     world, rank, local = dist_env()
@@ -748,7 +789,7 @@ def main():
     dev = torch.device("cuda", local)
     if args.mode != "decode":
         {"prefill": mode_prefill, "ablation": mode_ablation, "sweep": mode_sweep,
-         "docprefill": mode_docprefill,
+         "docprefill": mode_docprefill, "longanswer": mode_longanswer,
          "siblingscan": lambda *a: mode_ablation(*a, sibling=True)}[args.mode](
             args, world, rank, local, dev)
         if world > 1:

@@ -119,6 +119,13 @@ typedef struct pp_kv_layer {
  *                           (project page, section "More results"); same
  *                           result, kept to measure what per-stream segments
  *                           save.  Decode and question prefill only.
+ *   suffix_slices           decode suffix pass, how its warps share the (row,
+ *                           head) items: 0 = automatic (balanced when there
+ *                           are few items or segments may pass 512 keys),
+ *                           1 = equal item counts, 2 = balanced by work (an
+ *                           item longer than 8 chunks may be cut between
+ *                           warps; needs the tensor-core document pass and
+ *                           at most 4096 rows, else 1).  Same result.
  */
 typedef struct pp_options {
     int32_t splits;
@@ -127,6 +134,7 @@ typedef struct pp_options {
     int32_t wait_limit_log2;
     void **events;
     int32_t sibling_scan;
+    int32_t suffix_slices;
 } pp_options;
 
 /* Human-readable name of a pp_status value. */

@@ -97,19 +97,25 @@ SplitPlan plan_for(int rows, int H, int doc_len, const pp_options* opt, bool cau
 }
 
 struct WsLayout {
-  size_t doc_o, doc_ml, row_len, total;
+  size_t doc_o, doc_ml, row_len, split_cnt, split_o, split_ml, total;
 };
 
-// The document pass leaves its partial results in the workspace and, in a
-// decode step whose append it carries, each row's stream length (one int per
-// row; not needed by the causal document prefill).
+// The document pass leaves its partial results in the workspace.  Besides,
+// for decode and question prefill (not the causal document prefill): each
+// row's stream length when the pass carries a decode step's append, and the
+// decode suffix pass's counters and partials for items cut between warps.
 WsLayout ws_layout(const SplitPlan& p, int d) {
   WsLayout w;
   const size_t slots = (size_t)p.units * p.max_chunks * pp::kGroupRows;
+  const bool extra = slots && !p.causal;
+  const size_t warps = extra ? (size_t)std::max(sm_count(), 0) * pp::kSuffixWarps : 0;
   w.doc_o = 0;
   w.doc_ml = w.doc_o + up(slots * d * sizeof(float));
   w.row_len = w.doc_ml + up(slots * 2 * sizeof(float));
-  w.total = w.row_len + (slots && !p.causal ? up((size_t)p.G * pp::kGroupRows * sizeof(int32_t)) : 0);
+  w.split_cnt = w.row_len + (extra ? up((size_t)p.G * pp::kGroupRows * sizeof(int32_t)) : 0);
+  w.split_o = w.split_cnt + up(warps * sizeof(int32_t));
+  w.split_ml = w.split_o + up(2 * warps * d * sizeof(float));
+  w.total = w.split_ml + up(2 * warps * 2 * sizeof(float));
   return w;
 }
 
@@ -154,6 +160,7 @@ pp_status attend(const pp_kv_layer* L, int32_t doc_len, const uint16_t* q, const
   if (!causal && (!q_sid || !q_pos || !aligned(q_sid, 2) || !aligned(q_pos, 4)))
     return PP_ERR_INVALID_ARG;
   if (!(scale == scale)) return PP_ERR_INVALID_ARG;
+  if (opt && (opt->suffix_slices < 0 || opt->suffix_slices > 2)) return PP_ERR_INVALID_ARG;
   if (causal && opt && (opt->ablation_doc_per_stream || opt->sibling_scan))
     return PP_ERR_UNSUPPORTED;
   const SplitPlan plan = plan_for(rows, L->H, doc_len, opt, causal);
@@ -178,11 +185,26 @@ pp_status attend(const pp_kv_layer* L, int32_t doc_len, const uint16_t* q, const
                : cudaEventRecord(ev[i], st);
   };
   const bool other_doc = opt && (opt->ablation_doc_per_stream || opt->sibling_scan);
+  // decode behind the tensor-core document pass: the suffix slices are
+  // balanced by work, with counters that pass zeroes
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  pp::SuffixSplit split{};
+  // automatic: when equal item counts would leave warps idle (fewer items
+  // than twice the warps) or a few long segments could hold most of the work
+  const int slices = opt ? opt->suffix_slices : 0;
+  const bool want = slices == 2 ||
+                    (slices == 0 && ((int64_t)rows * L->H < 2LL * sms * pp::kSuffixWarps ||
+                                     L->S_cap > 32 * 16));
+  const bool balance = want && read_once && has_doc && !other_doc && rows <= pp::kBalanceRows;
+  if (balance) {
+    split.cnt = reinterpret_cast<int32_t*>(wsb + w.split_cnt);
+    split.o = reinterpret_cast<float*>(wsb + w.split_o);
+    split.ml = reinterpret_cast<float*>(wsb + w.split_ml);
+  }
   pp::AppendJob app{};
   if (app_k) {
     if (has_doc && !other_doc && rows <= kFusedAppendMaxRows) {
-      app = {app_k, app_v, q_sid, q_pos, rows,
-             reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + w.row_len)};
+      app = {app_k, app_v, q_sid, q_pos, rows, reinterpret_cast<int32_t*>(wsb + w.row_len)};
     } else if ((s = from_cuda(pp::launch_kv_append(*L, app_k, app_v, q_sid, q_pos, rows, st,
                                                    true))) != PP_OK) {
       return s;
@@ -195,7 +217,8 @@ pp_status attend(const pp_kv_layer* L, int32_t doc_len, const uint16_t* q, const
       e = pp::launch_doc_per_stream(*L, doc_len, q, rows, scale, plan.max_chunks, part, st);
     else
       e = pp::launch_doc_pass_tc(*L, doc_len, q, rows, scale, plan, part, wait_limit(opt),
-                                 opt ? opt->debug_inject_timeout : 0, app, st);
+                                 opt ? opt->debug_inject_timeout : 0, app, split.cnt,
+                                 balance ? sms * pp::kSuffixWarps : 0, st);
     if (e != cudaSuccess) return PP_ERR_CUDA;
   }
   if (mark(1) != cudaSuccess) return PP_ERR_CUDA;
@@ -206,7 +229,8 @@ pp_status attend(const pp_kv_layer* L, int32_t doc_len, const uint16_t* q, const
   } else if (read_once) {
     if ((s = from_cuda(pp::launch_suffix_merge(*L, q, q_sid, q_pos, rows, scale, plan, has_doc,
                                                part, o, lse, wait_limit(opt), sms,
-                                               app.n ? app.row_len : nullptr, st))) != PP_OK)
+                                               app.n ? app.row_len : nullptr,
+                                               balance ? &split : nullptr, st))) != PP_OK)
       return s;
   } else if ((s = from_cuda(pp::launch_suffix_block(*L, q, q_sid, q_pos, rows, scale, plan,
                                                     has_doc, part, o, lse, sms, st))) != PP_OK) {

@@ -197,6 +197,17 @@ struct Partials {
   float* doc_ml;    // [units*max_chunks][kGroupRows][2]  (max, sum), log2 domain
 };
 
+// Decode suffix pass: warps per CTA, and the largest row count it balances
+// by work (see suffix.cu); its scratch for items cut between warps.
+constexpr int kSuffixWarps = 12;
+constexpr int kBalanceRows = 4096;
+constexpr int kSnapUnits = 8;     // items of at most this many chunks are never cut
+struct SuffixSplit {
+  int32_t* cnt;     // [num_sms * kSuffixWarps] arrival counters, zeroed by the document pass
+  float* o;         // [2 * num_sms * kSuffixWarps][d]
+  float* ml;        // [2 * num_sms * kSuffixWarps][2]
+};
+
 // A decode step's append, carried out by one otherwise idle warp of each CTA
 // of the document pass (append_warp.cuh).  n = 0: nothing to append.
 struct AppendJob {

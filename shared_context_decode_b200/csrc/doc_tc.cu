@@ -66,6 +66,8 @@ struct DocTcParams {
   int inject_timeout;
   AppendJob app;  // a decode step's append, done by warp 2 (n = 0: none)
   pp_kv_layer L;
+  int32_t* zero;  // n_zero ints warp 2 sets to 0 (the suffix pass's counters)
+  int n_zero;
 };
 
 template <int D>
@@ -408,6 +410,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 2) {
     // ------------------------------- TMEM owner; idle until the teardown ----
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLow));
+    for (int i = blockIdx.x * 32 + lane; i < p.n_zero; i += gridDim.x * 32) p.zero[i] = 0;
     if (p.app.n > 0) append_pairs_warp<D>(p.app, p.L, blockIdx.x, gridDim.x, lane);
   } else {
     // ---------------------------------------------------------- softmax ----
@@ -638,7 +641,8 @@ namespace {
 template <int D>
 cudaError_t launch_impl(const pp_kv_layer& L, int doc_len, const uint16_t* q, int rows, float scale,
                         const SplitPlan& plan, const Partials& part, long long wait_limit,
-                        int inject, const AppendJob& app, cudaStream_t st) {
+                        int inject, const AppendJob& app, int32_t* zero, int n_zero,
+                        cudaStream_t st) {
   using C = DocCfg<D>;
   CUtensorMap mQ, mK, mV;
   if (!make_tmap_bf16_3d(&mQ, q, D, L.H, rows, (uint64_t)D * 2, (uint64_t)L.H * D * 2, 64, 1, 128) ||
@@ -679,6 +683,8 @@ cudaError_t launch_impl(const pp_kv_layer& L, int doc_len, const uint16_t* q, in
   prm.inject_timeout = inject;
   prm.app = app;
   prm.L = L;
+  prm.zero = zero;
+  prm.n_zero = n_zero;
   doc_pass_tc<D><<<plan.C * prm.pair, kThreads, C::SMEM, st>>>(mQ, mK, mV, prm);
   return cudaGetLastError();
 }
@@ -688,12 +694,12 @@ cudaError_t launch_impl(const pp_kv_layer& L, int doc_len, const uint16_t* q, in
 cudaError_t launch_doc_pass_tc(const pp_kv_layer& L, int doc_len, const uint16_t* q, int rows,
                                float scale, const SplitPlan& plan, const Partials& part,
                                long long wait_limit, int inject_timeout, const AppendJob& app,
-                               cudaStream_t st) {
+                               int32_t* zero, int n_zero, cudaStream_t st) {
   if (L.d == 128)
     return launch_impl<128>(L, doc_len, q, rows, scale, plan, part, wait_limit, inject_timeout,
-                            app, st);
+                            app, zero, n_zero, st);
   return launch_impl<64>(L, doc_len, q, rows, scale, plan, part, wait_limit, inject_timeout, app,
-                         st);
+                         zero, n_zero, st);
 }
 
 }  // namespace pp

@@ -11,6 +11,7 @@ namespace pp {
 
 struct SplitPlan;
 struct Partials;
+struct SuffixSplit;
 
 // 3-D bf16 TMA tensor map with 128-byte swizzle (zero fill out of range);
 // dims innermost first, strides of dims 1 and 2 in bytes.
@@ -31,10 +32,11 @@ cudaError_t launch_kv_reset_streams(const pp_kv_layer& L, const int16_t* sid, in
 
 // Document pass on the tensor cores; tensor maps are built inside.  app: a
 // decode step's append, done inside the launch (app.n = 0: none).
+// zero, n_zero: ints the launch sets to 0 (the suffix pass's counters).
 cudaError_t launch_doc_pass_tc(const pp_kv_layer& L, int doc_len, const uint16_t* q, int rows,
                                float scale, const SplitPlan& plan, const Partials& part,
                                long long wait_limit, int inject_timeout, const AppendJob& app,
-                               cudaStream_t st);
+                               int32_t* zero, int n_zero, cudaStream_t st);
 cudaError_t launch_doc_per_stream(const pp_kv_layer& L, int doc_len, const uint16_t* q, int rows,
                                   float scale, int max_chunks, const Partials& part,
                                   cudaStream_t st);
@@ -47,12 +49,14 @@ cudaError_t launch_sibling_scan(const pp_kv_layer& L, const uint16_t* q, const i
 // Suffix pass of a decode step (one warp per row and head) with the
 // log-sum-exp merge in its epilogue; writes o and lse.  row_len: the stream
 // lengths left by an append inside the document pass, per row (stored into
-// len by this kernel); nullptr: read len.
+// len by this kernel); nullptr: read len.  split: scratch whose counters the
+// document pass zeroed, for slices balanced by work (up to kBalanceRows
+// rows); nullptr: equal item counts per warp.
 cudaError_t launch_suffix_merge(const pp_kv_layer& L, const uint16_t* q, const int16_t* q_sid,
                                 const int32_t* q_pos, int rows, float scale, const SplitPlan& plan,
                                 bool has_doc, const Partials& part, uint16_t* o, float* lse,
                                 long long wait_limit, int num_sms, const int32_t* row_len,
-                                cudaStream_t st);
+                                const SuffixSplit* split, cudaStream_t st);
 // Suffix pass of a prefill call (one warp per 16 rows and head, warp-level
 // mma), merge first; q_sid = nullptr for document rows.  Writes o and lse.
 cudaError_t launch_suffix_block(const pp_kv_layer& L, const uint16_t* q, const int16_t* q_sid,

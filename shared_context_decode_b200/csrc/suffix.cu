@@ -7,10 +7,20 @@
 // every segment is read by one row); prefill calls, whose rows share their
 // question's segment, run the question-block kernel of suffix_block.cu.
 //
-// Work item = (query row, head).  Each warp owns a contiguous, balanced block
-// of items and a ring of NS shared-memory stages; lane 0 fills them with 1-D
+// Work item = (query row, head).  Each warp owns a contiguous slice of the
+// items and a ring of NS shared-memory stages; lane 0 fills them with 1-D
 // bulk copies of exactly the live keys of a chunk (a segment's rows are
 // contiguous), NS-1 chunks ahead of the warp and across item boundaries.
+//
+// Balance: segments differ in length (questions and answers of different
+// lengths), so equal item counts per warp leave the slowest warp with far
+// more chunks than the mean.  With up to kBalanceRows rows each CTA first
+// counts every item's work in units (its chunks, at least one for the merge)
+// and the warps take equal slices of the head-major unit sequence.  An item
+// cut by a slice boundary gets a partial (m, l, o) from each warp it spans;
+// each writes its partial, counts itself in the item's arrival counter
+// (zeroed by the document pass), and the last to arrive folds the others in
+// and finishes the item.  No warp waits for another.
 //
 // Scores: 8 lanes per key, each lane a 16-byte group g of every 128 bytes of
 // the row, so the 8 lanes of a shared-memory phase read one contiguous
@@ -35,7 +45,8 @@
 
 namespace pp {
 
-template <int D>
+// BAL: slices balanced by work (see above); false: equal item counts.
+template <int D, bool BAL = false>
 struct SufCfg {
   static constexpr int CK = 16;              // keys per chunk (8 or 16)
   static constexpr int NPASS = CK / 4;       // score passes of 4 keys
@@ -43,12 +54,14 @@ struct SufCfg {
   static constexpr int HALF = CK * ROWB;     // K (or V) part of a stage
   static constexpr int STAGE = 2 * HALF;
   static constexpr int NS = 2;               // stages per warp (NS-1 chunks in flight)
-  static constexpr int WARPS = 12;           // warps per CTA
-  static constexpr int TBL = 128;            // item-table entries per warp and round
+  static constexpr int WARPS = kSuffixWarps;  // warps per CTA
+  static constexpr int TBL = BAL ? 32 : 128;  // item-table entries per warp and round
   static constexpr int PRE = 4;              // document partials prefetched per lane
   static constexpr int G = D / 64;           // 16-byte groups per lane and key row
   static constexpr int E = D / 32;           // output dims per lane
-  static constexpr int SMEM = WARPS * NS * STAGE + WARPS * TBL * 16 + 128;
+  static constexpr int TBL_BYTES = WARPS * TBL * (BAL ? 24 : 16);   // ItemRec tables
+  static constexpr int PRE_BYTES = BAL ? (kBalanceRows + 1) * 4 : 0;  // units prefix over rows
+  static constexpr int SMEM = WARPS * NS * STAGE + TBL_BYTES + PRE_BYTES + 128;
   static_assert(SMEM <= 227 * 1024, "dynamic shared memory above the per-CTA limit");
 };
 
@@ -74,13 +87,34 @@ struct SufParams {
   uint16_t* o;
   float* lse;
   long long wait_limit;
+  // balanced slices (null: equal item counts per warp): arrival counters
+  // [gridDim.x * WARPS] zeroed before the launch, partials [2 per warp]
+  int32_t* split_cnt;
+  float* split_o;   // [2 * warps][d]  un-normalised
+  float* split_ml;  // [2 * warps][2]  (max, sum), log2 domain
 };
 
 // Per-item record of the warp's table: stream id (0 when the row is not an
-// answer-stream query), query position, visible-segment length, raw stream id.
+// answer-stream query), query position, visible-segment length, raw stream
+// id; balanced slices add the keys [tb, te) of the segment this warp covers
+// (else the whole segment).
+template <bool BAL>
 struct ItemRec {
   int s, qp, n, raw;
+  __device__ int tb() const { return 0; }
+  __device__ int te() const { return n; }
+  __device__ void set_range(int, int) {}
+  __device__ void clamp_range() {}
 };
+template <>
+struct ItemRec<true> {
+  int s, qp, n, raw, tb_, te_;
+  __device__ int tb() const { return tb_; }
+  __device__ int te() const { return te_; }
+  __device__ void set_range(int b, int e) { tb_ = b; te_ = e; }
+  __device__ void clamp_range() { te_ = te_ < n ? te_ : n; }
+};
+static_assert(sizeof(ItemRec<false>) == 16 && sizeof(ItemRec<true>) == 24, "table entry size");
 
 // Online-softmax state fold: (m, l, a) <- (m, l, a) (+) (m2, l2, a2).
 __device__ __forceinline__ void fold(float& m, float& l, float (&a)[8], float m2, float l2,
@@ -136,9 +170,10 @@ __device__ __forceinline__ int key_lane(int kk) {
   return (kk & 3) * 8 + (kk >> 2) * (8 / NPASS);
 }
 
-template <int D>
-__global__ void __launch_bounds__(SufCfg<D>::WARPS * 32) suffix_merge(const SufParams p) {
-  using C = SufCfg<D>;
+template <int D, bool BAL>
+__global__ void __launch_bounds__(SufCfg<D, BAL>::WARPS * 32) suffix_merge(const SufParams p) {
+  using C = SufCfg<D, BAL>;
+  using Rec = ItemRec<BAL>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) &
                                              ~uintptr_t(127));
@@ -150,7 +185,7 @@ __global__ void __launch_bounds__(SufCfg<D>::WARPS * 32) suffix_merge(const SufP
   // key whose score this lane ends with
   const int my_key = C::NPASS == 4 ? 4 * (2 * b2 + b1) + sub : 4 * b2 + sub;
   uint8_t* ring = smem + warp * C::NS * C::STAGE;
-  ItemRec* tbl = reinterpret_cast<ItemRec*>(smem + C::WARPS * C::NS * C::STAGE) + warp * C::TBL;
+  Rec* tbl = reinterpret_cast<Rec*>(smem + C::WARPS * C::NS * C::STAGE) + warp * C::TBL;
   uint64_t* full = bars[warp];
   if (threadIdx.x == 0) abort_sh = 0;
   if (lane == 0) {
@@ -160,35 +195,119 @@ __global__ void __launch_bounds__(SufCfg<D>::WARPS * 32) suffix_merge(const SufP
   __syncthreads();
   volatile int* abort_flag = &abort_sh;
 
-  // This warp's items: a contiguous, balanced block of the (head, row) space,
-  // head-major, so in a prefill neighbouring items share a segment.
   const int64_t items = (int64_t)p.rows * p.H;
   const int64_t gw = (int64_t)blockIdx.x * C::WARPS + warp;
   const int64_t GW = (int64_t)gridDim.x * C::WARPS;
-  const int64_t i_begin = gw * items / GW, i_end = (gw + 1) * items / GW;
   const int groups = (p.rows + kGroupRows - 1) / kGroupRows;
-  // document prefill: no stream ids; row r is document token r and sees only
-  // the document (its partials carry the causal mask)
-  const bool doc_rows = p.q_sid == nullptr;
   const size_t seg_elems = (size_t)p.S_cap * D;
+  constexpr bool balanced = BAL;
+
+  // Units of row r (every head alike): max(1, chunks of its visible
+  // segment); pre[r] = units of rows 0 .. r-1.
+  int32_t* pre = reinterpret_cast<int32_t*>(smem + C::WARPS * C::NS * C::STAGE + C::TBL_BYTES);
+  int64_t T = 0;       // units of all items
+  int Ctot = 1;        // units of one head's rows
+  if constexpr (balanced) {
+    for (int r = threadIdx.x; r < p.rows; r += blockDim.x) {
+      const int s = p.q_sid[r];
+      int n = 0;
+      if (stream_query(s, p.P_max)) {
+        n = p.row_len ? p.row_len[r] : p.len[s - 1];
+        n = n < p.S_cap ? n : p.S_cap;
+      }
+      pre[r + 1] = n > C::CK ? (n + C::CK - 1) / C::CK : 1;
+    }
+    if (threadIdx.x == 0) pre[0] = 0;
+    __syncthreads();
+    // in-place inclusive scan of pre[1 .. rows]: runs per thread, then an
+    // exclusive scan of the run totals across the block
+    __shared__ int wsum[C::WARPS];
+    const int per = (p.rows + (int)blockDim.x - 1) / (int)blockDim.x;
+    const int b = (int)threadIdx.x * per + 1;
+    const int e = min(b + per, p.rows + 1);
+    int run = 0;
+    for (int i = b; i < e; ++i) {
+      run += pre[i];
+      pre[i] = run;
+    }
+    int x = run;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane == 31) wsum[warp] = x;
+    __syncthreads();
+    int off = x - run;
+    for (int w2 = 0; w2 < warp; ++w2) off += wsum[w2];
+    for (int i = b; i < e; ++i) pre[i] += off;
+    __syncthreads();
+    Ctot = pre[p.rows];
+    T = (int64_t)Ctot * p.H;
+  }
+  // slices over min(GW, T) warps, so none is empty (warps past it idle)
+  const int64_t GWe = T < GW ? T : GW;
+  // item holding unit u: head u / Ctot, then the last row whose prefix is <= the rest
+  auto item_of = [&](int64_t u) -> int64_t {
+    const int h = (int)(u / Ctot);
+    const int x = (int)(u - (int64_t)h * Ctot);
+    int lo = 0, hi = p.rows - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (pre[mid] <= x) lo = mid; else hi = mid - 1;
+    }
+    return (int64_t)h * p.rows + lo;
+  };
+  // warp whose slice holds unit u (slice w = [w T / GWe, (w + 1) T / GWe))
+  auto warp_of = [&](int64_t u) -> int64_t { return ((u + 1) * GWe - 1) / T; };
+  // A slice boundary inside an item of at most kSnapUnits units moves to
+  // the nearer edge of the item: only long items are cut (their interior
+  // boundaries stay where they are, so warp_of still finds their warps).
+  auto snap = [&](int64_t u) -> int64_t {
+    if (u <= 0 || u >= T) return u;
+    const int64_t it = item_of(u);
+    const int r = (int)(it % p.rows);
+    const int64_t S = (it / p.rows) * Ctot + pre[r];
+    const int U = pre[r + 1] - pre[r];
+    if (u == S || U > kSnapUnits) return u;
+    return (u - S) * 2 <= U ? S : S + U;
+  };
+  // this warp's items, first .. last inclusive, and (balanced) its units
+  int64_t i_first, i_last, u_lo = 0, u_hi = 0;
+  if constexpr (balanced) {
+    u_lo = gw < GWe ? snap(gw * T / GWe) : 0;
+    u_hi = gw < GWe ? snap((gw + 1) * T / GWe) : 0;
+    i_first = u_lo < u_hi ? item_of(u_lo) : 0;
+    i_last = u_lo < u_hi ? item_of(u_hi - 1) : -1;
+  } else {
+    i_first = gw * items / GW;
+    i_last = (gw + 1) * items / GW - 1;
+  }
 
   // each segment is read once, so its lines go first and the document
   // partials the merge reads stay in L2
   const uint64_t pol = l2_policy_evict_first();
   uint32_t issued = 0, consumed = 0;
   bool ok = true;
-  for (int64_t r0 = i_begin; ok && r0 < i_end; r0 += C::TBL) {
-    const int cnt = (int)min((int64_t)C::TBL, i_end - r0);
+  for (int64_t r0 = i_first; ok && r0 <= i_last; r0 += C::TBL) {
+    const int cnt = (int)min((int64_t)C::TBL, i_last - r0 + 1);
     // ---- item table of this round: two parallel gathers instead of one
     // dependent chain per item
     for (int k = lane; k < cnt; k += 32) {
-      const int r = (int)((r0 + k) % p.rows);
-      const int s = doc_rows ? 0 : p.q_sid[r];
-      ItemRec rec;
-      rec.qp = doc_rows ? r : p.q_pos[r];
+      const int64_t item = r0 + k;
+      const int r = (int)(item % p.rows);
+      const int s = p.q_sid[r];
+      Rec rec;
+      rec.qp = p.q_pos[r];
       rec.s = stream_query(s, p.P_max) ? s : 0;
       rec.n = 0;
       rec.raw = s;
+      if constexpr (balanced) {  // this warp's units of the item, as keys
+        const int64_t S = (item / p.rows) * Ctot + pre[r];
+        const int64_t U = pre[r + 1] - pre[r];
+        rec.set_range((int)((u_lo > S ? u_lo - S : 0) * C::CK),
+                      (int)((u_hi < S + U ? u_hi - S : U) * C::CK));
+      }
       tbl[k] = rec;
     }
     __syncwarp();
@@ -205,22 +324,23 @@ __global__ void __launch_bounds__(SufCfg<D>::WARPS * 32) suffix_merge(const SufP
         }
         tbl[k].n = n < p.S_cap ? n : p.S_cap;
       }
+      tbl[k].clamp_range();
     }
     __syncwarp();
 
     // Producer cursor over (item, first key) chunks of this round.
-    int pk = 0, pt0 = 0;
+    int pk = 0, pt0 = cnt > 0 ? tbl[0].tb() : 0;
     auto issue_next = [&](uint32_t stage) -> bool {
-      while (pk < cnt && pt0 >= tbl[pk].n) {
+      while (pk < cnt && pt0 >= tbl[pk].te()) {
         ++pk;
-        pt0 = 0;
+        pt0 = pk < cnt ? tbl[pk].tb() : 0;
       }
       if (pk >= cnt) return false;
       if (lane == 0) {
-        const ItemRec rec = tbl[pk];
+        const Rec rec = tbl[pk];
         const int h = (int)((r0 + pk) / p.rows);
         const size_t seg = ((size_t)(rec.s - 1) * p.H + h) * seg_elems + (size_t)pt0 * D;
-        const int nk = min(C::CK, rec.n - pt0);
+        const int nk = min(C::CK, rec.te() - pt0);
         uint8_t* st = ring + stage * C::STAGE;
         fence_proxy_async();
         mbar_arrive_expect_tx(full + stage, 2u * nk * C::ROWB);
@@ -243,12 +363,12 @@ __global__ void __launch_bounds__(SufCfg<D>::WARPS * 32) suffix_merge(const SufP
       const uint4* qp4 = reinterpret_cast<const uint4*>(p.q + ((int64_t)r * p.H + h) * D);
 #pragma unroll
       for (int c = 0; c < C::G; ++c) qn[c] = __ldg(qp4 + g + 8 * c);
-      const ItemRec rec = tbl[k];
+      const Rec rec = tbl[k];
       sid0 = -1;
       pos0 = 0;
-      if (my_key < rec.n) {
-        sid0 = __ldg(p.sid + (size_t)(rec.s - 1) * p.S_cap + my_key);
-        pos0 = __ldg(p.pos + (size_t)(rec.s - 1) * p.S_cap + my_key);
+      if (rec.tb() + my_key < rec.te()) {
+        sid0 = __ldg(p.sid + (size_t)(rec.s - 1) * p.S_cap + rec.tb() + my_key);
+        pos0 = __ldg(p.pos + (size_t)(rec.s - 1) * p.S_cap + rec.tb() + my_key);
       }
     };
     if (cnt > 0) prefetch_item(0);
@@ -256,14 +376,14 @@ __global__ void __launch_bounds__(SufCfg<D>::WARPS * 32) suffix_merge(const SufP
     for (int k = 0; k < cnt; ++k) {
       const int64_t item = r0 + k;
       const int h = (int)(item / p.rows), r = (int)(item - (int64_t)h * p.rows);
-      const ItemRec rec = tbl[k];
+      const Rec rec = tbl[k];
       uint4 qr[C::G];
 #pragma unroll
       for (int c = 0; c < C::G; ++c) qr[c] = qn[c];
       // this lane's key tags, loaded one chunk ahead of their use
       int nsid = sid0, npos = pos0;
       if (k + 1 < cnt) prefetch_item(k + 1);
-      const bool valid = rec.s != 0 || doc_rows;
+      const bool valid = rec.s != 0;
       // document partials of this (row, head), fetched now so their latency
       // hides behind the segment's chunks
       int c0 = 0, c1 = -1;
@@ -314,12 +434,12 @@ __global__ void __launch_bounds__(SufCfg<D>::WARPS * 32) suffix_merge(const SufP
       const int16_t* sb = p.sid + (size_t)(valid ? rec.s - 1 : 0) * p.S_cap;
       const int32_t* pb = p.pos + (size_t)(valid ? rec.s - 1 : 0) * p.S_cap;
 
-      for (int t0 = 0; t0 < rec.n; t0 += C::CK) {
+      for (int t0 = rec.tb(); t0 < rec.te(); t0 += C::CK) {
         if (issue_next(issued % C::NS)) ++issued;
         const int t = t0 + my_key;
         const int tsid = nsid, tpos = npos;
         nsid = -1;
-        if (t + C::CK < rec.n) {
+        if (t + C::CK < rec.te()) {
           nsid = __ldg(sb + t + C::CK);
           npos = __ldg(pb + t + C::CK);
         }
@@ -375,7 +495,7 @@ __global__ void __launch_bounds__(SufCfg<D>::WARPS * 32) suffix_merge(const SufP
           dot += __shfl_xor_sync(0xffffffffu, dot, 2);
         }
         dot += __shfl_xor_sync(0xffffffffu, dot, 1);
-        const float x = slot_visible(rec.s, rec.qp, tsid, tpos, t, rec.n) ? dot : -INFINITY;
+        const float x = slot_visible(rec.s, rec.qp, tsid, tpos, t, rec.te()) ? dot : -INFINITY;
         // chunk maximum over the lanes holding distinct keys
         float cm = fmaxf(m, x);
 #pragma unroll
@@ -424,6 +544,50 @@ __global__ void __launch_bounds__(SufCfg<D>::WARPS * 32) suffix_merge(const SufP
         for (int e = 0; e < C::E; ++e) acc[e] = acc[e] * xa + a2[e] * ya;
         m = mm;
       };
+      if constexpr (balanced) {
+        // an item cut by slice boundaries: publish this warp's partial; the
+        // last of its warps to arrive folds the others in and finishes it
+        const int64_t S = (int64_t)h * Ctot + pre[r];
+        const int U = pre[r + 1] - pre[r];
+        const int64_t wf = warp_of(S), wl = warp_of(S + U - 1);
+        if (U > kSnapUnits && wf != wl) {
+          // partial slot: 2 w for the warp's first item, 2 w + 1 for its last
+          const int64_t slot = 2 * gw + (item == i_first ? 0 : 1);
+#pragma unroll
+          for (int e = 0; e < C::E; ++e) __stcg(p.split_o + slot * D + lane * C::E + e, acc[e]);
+          if (lane == 0) __stcg(reinterpret_cast<float2*>(p.split_ml) + slot, make_float2(m, l));
+          __threadfence();
+          __syncwarp();
+          int old = 0;
+          if (lane == 0) old = atomicAdd(p.split_cnt + wf, 1);
+          old = __shfl_sync(0xffffffffu, old, 0);
+          if (old != (int)(wl - wf)) continue;  // not the last: another warp finishes the item
+          __threadfence();
+          // fold every warp's partial in warp order, so the result does not
+          // depend on which warp arrived last
+          const float m_own = m, l_own = l;
+          float a_own[C::E];
+#pragma unroll
+          for (int e = 0; e < C::E; ++e) {
+            a_own[e] = acc[e];
+            acc[e] = 0.f;
+          }
+          m = -INFINITY;
+          l = 0.f;
+          for (int64_t w2 = wf; w2 <= wl; ++w2) {
+            if (w2 == gw) {
+              fold_in(m_own, l_own, a_own);
+              continue;
+            }
+            const int64_t s2 = 2 * w2 + ((w2 == wf && snap(w2 * T / GWe) < S) ? 1 : 0);
+            const float2 ml = __ldcg(reinterpret_cast<const float2*>(p.split_ml) + s2);
+            float a2[C::E];
+#pragma unroll
+            for (int e = 0; e < C::E; ++e) a2[e] = __ldcg(p.split_o + s2 * D + lane * C::E + e);
+            fold_in(ml.x, ml.y, a2);
+          }
+        }
+      }
 #pragma unroll
       for (int e = 0; e < C::PRE; ++e)
         if (c0 + e <= c1) fold_in(pre_ml[e].x, pre_ml[e].y, pre_o[e]);
@@ -448,7 +612,7 @@ __global__ void __launch_bounds__(SufCfg<D>::WARPS * 32) suffix_merge(const SufP
       }
       if (lane == 0) {
         if (p.lse) p.lse[(int64_t)r * p.H + h] = any ? (m + log2f(l)) * kLn2 : -INFINITY;
-        if (h == 0 && !doc_rows && (rec.raw == 0 || rec.raw > p.P_max))
+        if (h == 0 && (rec.raw == 0 || rec.raw > p.P_max))
           set_status(p.status, PP_DEV_BAD_STREAM);
       }
     }
@@ -466,8 +630,12 @@ cudaError_t launch_suffix_merge(const pp_kv_layer& L, const uint16_t* q, const i
                                 const int32_t* q_pos, int rows, float scale, const SplitPlan& plan,
                                 bool has_doc, const Partials& part, uint16_t* o, float* lse,
                                 long long wait_limit, int num_sms, const int32_t* row_len,
-                                cudaStream_t st) {
+                                const SuffixSplit* split, cudaStream_t st) {
   SufParams prm;
+  const bool bal = split && rows <= kBalanceRows;
+  prm.split_cnt = bal ? split->cnt : nullptr;
+  prm.split_o = bal ? split->o : nullptr;
+  prm.split_ml = bal ? split->ml : nullptr;
   prm.rows = rows;
   prm.H = L.H;
   prm.P_max = L.P_max;
@@ -506,9 +674,13 @@ cudaError_t launch_suffix_merge(const pp_kv_layer& L, const uint16_t* q, const i
     kernel<<<(int)ctas, warps * 32, smem, st>>>(prm);
     return cudaGetLastError();
   };
-  static std::atomic<uint64_t> ready128{0}, ready64{0};
-  if (L.d == 128) return go(suffix_merge<128>, SufCfg<128>::WARPS, SufCfg<128>::SMEM, ready128);
-  return go(suffix_merge<64>, SufCfg<64>::WARPS, SufCfg<64>::SMEM, ready64);
+  static std::atomic<uint64_t> ready[4];
+  if (L.d == 128)
+    return bal ? go(suffix_merge<128, true>, SufCfg<128, true>::WARPS, SufCfg<128, true>::SMEM,
+                    ready[0])
+               : go(suffix_merge<128, false>, SufCfg<128>::WARPS, SufCfg<128>::SMEM, ready[1]);
+  return bal ? go(suffix_merge<64, true>, SufCfg<64, true>::WARPS, SufCfg<64, true>::SMEM, ready[2])
+             : go(suffix_merge<64, false>, SufCfg<64>::WARPS, SufCfg<64>::SMEM, ready[3]);
 }
 
 // K6 (ablation): the document read once PER QUERY ROW -- one warp per (row,

@@ -44,7 +44,8 @@ class LayerStruct(ctypes.Structure):
 class Options(ctypes.Structure):
     _fields_ = [("splits", _i32), ("ablation_doc_per_stream", _i32),
                 ("debug_inject_timeout", _i32), ("wait_limit_log2", _i32),
-                ("events", ctypes.POINTER(_vp)), ("sibling_scan", _i32)]
+                ("events", ctypes.POINTER(_vp)), ("sibling_scan", _i32),
+                ("suffix_slices", _i32)]
 
     def set_events(self, events):
         """Record 3 CUDA events (torch.cuda.Event, enable_timing=True) around

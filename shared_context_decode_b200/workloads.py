@@ -40,6 +40,9 @@ CONFIGS = {
     "doc8k_p64": dict(layers=32, H=32, d=128, N=8192, P=64, q=(16, 48), a=(0, 31)),
     # same shapes, doc 16384, 256 streams: the memory-bound headline case
     "doc16k_p256": dict(layers=32, H=32, d=128, N=16384, P=256, q=(16, 48), a=(0, 63)),
+    # long answers: doc 8192, 128 streams, 1024 answer tokens already cached
+    # (the long-answer point of the pages' answer-length figure)
+    "doc8k_p128_a1k": dict(layers=8, H=32, d=128, N=8192, P=128, q=(16, 48), a=(1024, 1024)),
     # question prefill: doc 12000 cached, 256 questions of 16..48 tokens
     "prefill_doc12k_p256": dict(layers=32, H=32, d=128, N=12000, P=256, q=(16, 48),
                                 a=(0, 0)),

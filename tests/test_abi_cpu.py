@@ -78,6 +78,8 @@ def test_host_validation_codes(pp):
     assert call_decode(pp, L, P=0) == pp.PP_OK                        # empty: nothing launched
     opt = pp.Options(splits=4)
     assert call_decode(pp, L, ws_bytes=16, opt=opt) == pp.PP_ERR_CAPACITY
+    assert call_decode(pp, L, opt=pp.Options(suffix_slices=3)) == pp.PP_ERR_INVALID_ARG
+    assert call_decode(pp, L, opt=pp.Options(suffix_slices=-1)) == pp.PP_ERR_INVALID_ARG
     # append
     assert pp._kv_append(ctypes.byref(L), 0x1000, 0x2000, 0x3000, 0x4000, -1, None) == \
         pp.PP_ERR_INVALID_ARG

@@ -100,6 +100,57 @@ def test_full_size_sampled(name):
         decode_case(W, l=l, rows=rows)
 
 
+@pytest.mark.parametrize("P,H,q,a", [(3, 2, (10, 20), (1500, 2500)), (40, 2, (1, 30), (0, 600)),
+                                     (7, 1, (1, 1), (0, 0))])
+@pytest.mark.parametrize("slices", [0, 1, 2])
+def test_segments_split_between_warps(P, H, q, a, slices):
+    """Few streams with long segments: with work-balanced slices the suffix
+    pass cuts long items between warps, and the last warp of each item merges
+    the partials of the others; also one-key segments with more warps than
+    work.  Each slicing of the work gives the oracle's result."""
+    m = gu.pp()
+    W = wl.make_decode(layers=1, H=H, d=128, N=700, P=P, q=q, a=a, seed=21, device=DEV)
+    decode_case(W, opt=m.Options(suffix_slices=slices))
+
+
+@pytest.mark.parametrize("slices", [1, 2])
+def test_ragged_rows_both_slicings(slices):
+    m = gu.pp()
+    W = wl.make_decode(layers=1, H=4, d=64, N=1000, P=200, q=(1, 20), a=(0, 90), seed=23,
+                       device=DEV)
+    decode_case(W, opt=m.Options(suffix_slices=slices))
+
+
+def test_split_items_replayed_in_a_graph_stay_exact():
+    """The arrival counters are zeroed by the document pass of every call:
+    repeated graph replays give identical outputs."""
+    m = gu.pp()
+    W = wl.make_decode(layers=1, H=2, d=128, N=500, P=5, q=(5, 9), a=(300, 700), seed=22,
+                       device=DEV)
+    L = W.layer(0)
+    layer = gu.load_decode(W, L, DEV)
+    o = torch.empty_like(L.q)
+    ws = m.workspace(m.decode_workspace_bytes(W.P, W.H, W.d, W.N), DEV)
+    opt = m.Options(suffix_slices=2)
+    m.decode_attn(layer, W.N, L.q, L.q_sid, L.q_pos, W.scale, o=o, ws=ws, opt=opt)
+    torch.cuda.synchronize()
+    first = o.clone()
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            m.decode_attn(layer, W.N, L.q, L.q_sid, L.q_pos, W.scale, o=o, ws=ws, opt=opt)
+    torch.cuda.current_stream().wait_stream(s)
+    for _ in range(5):
+        o.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(o.view(torch.int16), first.view(torch.int16))
+    o_ref, lse_ref, _ = gu.oracle_decode(W, L)
+    gu.compare(first, None, o_ref, None, "split items")
+
+
 def test_prefill_small_full():
     m = gu.pp()
     W = wl.make_prefill(layers=1, H=2, d=128, N=700, P=12, q=(1, 40), seed=9, device=DEV)
