@@ -669,7 +669,7 @@ def measure_doc_pass(step: DecodeStep, reps: int):
     opts = []
     for l in range(step.layers):
         o = pp.Options()
-        if step.opts is not None:   # same kernels as the timed step, plus the events
+        if getattr(step, "opts", None) is not None:   # same kernels as the timed step, plus the events
             for f, _ in pp.Options._fields_:
                 if f != "events":
                     setattr(o, f, getattr(step.opts[l], f))
