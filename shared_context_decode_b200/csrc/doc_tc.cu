@@ -89,7 +89,9 @@ struct DocCfg {
   static constexpr int SMEM = (USED + 1024) > 120 * 1024 ? (USED + 1024) : 120 * 1024;
   // the per-CTA limit covers the static exchange buffer (4 KB) as well
   static_assert(SMEM + 4352 <= 227 * 1024, "shared memory above the per-CTA limit");
-  static constexpr uint32_t T_O = 0, T_S = D;        // S buffer b at T_S + b * kBN
+  // O_0 | O_1 | S_0 | S_1: O_h accumulates the keys of column half h of
+  // every tile (each half keeps its own running maximum and sum)
+  static constexpr uint32_t T_O = 0, T_S = 2 * D;    // O_h at T_O + h * D, S_b at T_S + b * kBN
   static constexpr uint32_t TMEM_COLS = 512;
   static_assert(T_S + 2 * kBN <= TMEM_COLS, "TMEM budget");
   static_assert(kBN == 128, "one TMA box of keys per tile");
@@ -328,15 +330,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (elect_one()) mma_ss(d_t, dQ + off, b0 + off, IDESC_QK, kk > 0 ? 1u : 0u);
       }
     };
+    // O_h += P_h V_h for the two column halves of the tile: P_h (64 keys,
+    // bf16 pairs) sits in the first 32 columns of half h's part of S_b.
     auto issue_pv = [&](int b, int vslot, bool acc) {
-      const uint32_t d_t = tmem + C::T_O;
-      const uint32_t a_t = tmem + C::T_S + (uint32_t)(b * kBN);
       const uint64_t b0 = dV + (uint64_t)((vslot * C::KV_STAGE) >> 4);
 #pragma unroll
-      for (int kk = 0; kk < kBN / 16; ++kk)
-        if (elect_one())
-          mma_ts(d_t, a_t + kk * 8, b0 + (uint64_t)((kk * 16 * 128) >> 4), IDESC_PV,
-                 (acc || kk > 0) ? 1u : 0u);
+      for (int h = 0; h < 2; ++h) {
+        const uint32_t d_t = tmem + C::T_O + (uint32_t)(h * D);
+        const uint32_t a_t = tmem + C::T_S + (uint32_t)(b * kBN + h * (kBN / 2));
+#pragma unroll
+        for (int kk = 0; kk < kBN / 32; ++kk)
+          if (elect_one())
+            mma_ts(d_t, a_t + kk * 8, b0 + (uint64_t)(((h * (kBN / 32) + kk) * 16 * 128) >> 4),
+                   IDESC_PV, (acc || kk > 0) ? 1u : 0u);
+      }
     };
     auto commit = [&](uint64_t* bar_) {
       if (elect_one()) tc_commit(bar_);
@@ -419,9 +426,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int wq = warp & 3;                 // TMEM lane quarter of this warp
     const int rt = wq * 32 + lane;           // row inside the M tile
     constexpr int HB = kBN / 2;              // columns of S per half
-    constexpr int OC = D / 64;               // 32-column chunks of O per half
+    constexpr int OC = D / 32;               // 32-column chunks of O_h
     const uint32_t t_lane = tmem + ((uint32_t)(wq * 32) << 16);
-    const uint32_t t_O = t_lane + C::T_O + hf * (D / 2);
+    const uint32_t t_O = t_lane + C::T_O + hf * D;   // this half's accumulator
     int64_t t = t_begin;
     Seg s;
     uint32_t s_ph = 0, od_ph = 0;  // s_ph bit b: parity of s_full[b]
@@ -459,7 +466,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     while (ok && next_seg(p, t, t_end, slot, mt, s)) {
       if (!s.active) continue;
-      float m = -INFINITY, l = 0.f;   // l: this half's share of the row sum
+      float m = -INFINITY, l = 0.f;   // this half's running maximum and sum
       for (int j = s.j0; j < s.j1; ++j, ++g) {
         const int b = (j - s.j0) & 1;
         const uint32_t t_S = t_lane + C::T_S + (uint32_t)(b * kBN);
@@ -493,24 +500,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < HB; i += 2)
           mc[(i >> 1) & 7] = fmax3(mc[(i >> 1) & 7], __uint_as_float(r[i >> 5][i & 31]),
                                    __uint_as_float(r[i >> 5][(i & 31) + 1]));
-        float mx = fmax3(fmax3(mc[0], mc[1], mc[2]), fmax3(mc[3], mc[4], mc[5]), fmaxf(mc[6], mc[7]));
-        // The swap also orders both halves' reads of S before either half's
-        // P overwrites columns the other half read.
-        float mo;
-        if (!(ok = swap_half(mx, mo))) break;
-        mx = fmaxf(mx, mo);
+        const float mx =
+            fmax3(fmax3(mc[0], mc[1], mc[2]), fmax3(mc[3], mc[4], mc[5]), fmaxf(mc[6], mc[7]));
         const float m_new = fmaxf(m, mx * p.sl2);
         // Lazy rescale: keep a stale maximum unless the new one exceeds it
-        // by more than 2^8 (probabilities then stay below 256).  Both halves
-        // see the same maximum and take the same decision.
+        // by more than 2^8 (probabilities then stay below 256).
         const bool need = m_new > m + 8.f;
         const float m_old = m;
         if (need) {
           l *= ex2_mufu(m - m_new);
           m = m_new;
         }
-        // P = 2^(S * scale*log2e - m) as bf16 pairs, written over the S
-        // buffer's first 64 columns (this half's 32 of them).
+        // P = 2^(S * scale*log2e - m) as bf16 pairs, written over the first
+        // 32 of this half's 64 S columns (only this thread read them).
         // (a row that has seen no key yet keeps m = -inf: its P is 0)
         const float mneg = m == -INFINITY ? 0.f : -m;
         const float2 sl2v = make_float2(p.sl2, p.sl2), negm = make_float2(mneg, mneg);
@@ -533,11 +535,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             rs[pr_i & 1] = fadd2(rs[pr_i & 1], pv);
             pk[e >> 1] = f2_to_bf2(pv.x, pv.y);
           }
-          tmem_st16(t_S + hf * (HB / 2) + c * 16, pk);
+          tmem_st16(t_S + hf * HB + c * 16, pk);
         }
         l += (rs[0].x + rs[0].y) + (rs[1].x + rs[1].y);
-        // O rescale for rows whose maximum moved (rare), this half's O
-        // columns.  The previous tile's O += P V may still run: wait for it
+        // O_h rescale for rows whose maximum moved (rare).  The previous tile's O += P V may still run: wait for it
         // (pv_done completes once per product, so its phase g - 1 is that
         // one); this tile's is not issued before p_full.
         if (j > s.j0 && __any_sync(0xffffffffu, need)) {
@@ -567,22 +568,37 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool valid = row < p.rows;
       const int64_t pslot = (int64_t)s.u * p.plan.max_chunks + s.chunk;
       const int64_t prow = pslot * kGroupRows + mt * 128 + rt;
+      // Combine the halves: M = max(m_0, m_1), O = sum_h O_h 2^(m_h - M),
+      // L = sum_h l_h 2^(m_h - M); this half writes output columns
+      // [hf D/2, (hf+1) D/2) from both accumulators.
+      float mo, lo;
+      if (!(ok = swap_half(m, mo)) || !(ok = swap_half(l, lo))) break;
+      const float mm = fmaxf(m, mo);
+      const float f_own = m == -INFINITY ? 0.f : ex2_mufu(m - mm);
+      const float f_oth = mo == -INFINITY ? 0.f : ex2_mufu(mo - mm);
+      const float f0 = hf == 0 ? f_own : f_oth, f1 = hf == 0 ? f_oth : f_own;
+      const uint32_t t_O0 = t_lane + C::T_O + hf * (D / 2), t_O1 = t_O0 + D;
       float4* dst = reinterpret_cast<float4*>(p.doc_o + prow * D + hf * (D / 2));
 #pragma unroll
-      for (int c = 0; c < OC; ++c) {
-        uint32_t o[32];
-        tmem_ld32(t_O + c * 32, o);
+      for (int c = 0; c < OC / 2; ++c) {
+        uint32_t o0[32], o1[32];
+        tmem_ld32(t_O0 + c * 32, o0);
+        tmem_ld32(t_O1 + c * 32, o1);
         tmem_ld_wait();
         if (valid) {
 #pragma unroll
-          for (int e = 0; e < 32; e += 4)
-            dst[(c * 32 + e) / 4] = make_float4(__uint_as_float(o[e]), __uint_as_float(o[e + 1]),
-                                                __uint_as_float(o[e + 2]), __uint_as_float(o[e + 3]));
+          for (int e = 0; e < 32; e += 4) {
+            float4 v;
+            v.x = __uint_as_float(o0[e]) * f0 + __uint_as_float(o1[e]) * f1;
+            v.y = __uint_as_float(o0[e + 1]) * f0 + __uint_as_float(o1[e + 1]) * f1;
+            v.z = __uint_as_float(o0[e + 2]) * f0 + __uint_as_float(o1[e + 2]) * f1;
+            v.w = __uint_as_float(o0[e + 3]) * f0 + __uint_as_float(o1[e + 3]) * f1;
+            dst[(c * 32 + e) / 4] = v;
+          }
         }
       }
-      float lo;
-      if (!(ok = swap_half(l, lo))) break;
-      if (valid && hf == 0) reinterpret_cast<float2*>(p.doc_ml)[prow] = make_float2(m, l + lo);
+      if (valid && hf == 0)
+        reinterpret_cast<float2*>(p.doc_ml)[prow] = make_float2(mm, l * f_own + lo * f_oth);
       tc_fence_before();
       mbar_arrive(B.o_free);
     }
