@@ -36,8 +36,7 @@
 //   lse = (M + log2 Lsum) ln 2,
 // the softmax over the union of the key sets in max-shifted form.  Rows that
 // are not answer-stream queries, and rows that see nothing, get o = 0 and
-// lse = -inf.  Called without stream ids (a document prefill), every row is a
-// document token: no segment keys, only its document partials.
+// lse = -inf.
 #include <atomic>
 
 #include "common.cuh"
