@@ -170,7 +170,9 @@ pp_status pp_kv_reset_streams(const pp_kv_layer *layer, const int16_t *sid, int3
  * the same stream in this call; its sid and pos are stored with it, and
  * len[s-1] advances.  A full segment drops the row and sets
  * PP_DEV_SEGMENT_OVERFLOW; sid > P_max sets PP_DEV_BAD_STREAM; sid < 0 rows
- * are skipped.  Two kernel launches; n = 0 launches nothing.
+ * are skipped.  Two rows of one call at the same document position: which
+ * of them lands is unspecified.  Two kernel launches; n = 0 launches
+ * nothing.
  */
 pp_status pp_kv_append(const pp_kv_layer *layer, const uint16_t *k, const uint16_t *v,
                        const int16_t *sid, const int32_t *pos, int32_t n, void *stream);

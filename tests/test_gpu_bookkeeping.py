@@ -51,6 +51,56 @@ def test_append_matches_replay_bit_exact():
     assert m.device_status(layer) == expect
 
 
+@pytest.mark.parametrize("n", [300, 3000, 20000])
+def test_large_mixed_calls_match_replay_bit_exact(n):
+    """Calls large enough that one CTA takes many rows (up to 64): stream,
+    document, inactive and out-of-range rows mixed, streams repeated, some
+    segments overflowing."""
+    m = gu.pp()
+    H, d, P_max, doc_cap = 1, 64, 37, 400
+    S_cap = max(8, n // (2 * P_max))
+    layer = m.KVLayer(H, d, doc_cap, P_max, S_cap, DEV)
+    m.kv_reset(layer)
+    R = AppendReplay(P_max, S_cap, doc_cap)
+    rng = np.random.default_rng(n)
+    for call in range(2):
+        sid = rng.integers(-1, P_max + 3, size=n).astype(np.int16)
+        pos = rng.integers(-2, doc_cap + 2, size=n).astype(np.int32)
+        # document rows of one call take distinct positions (two rows of a
+        # call at one document position are the caller's error)
+        doc_rows = np.nonzero(sid == 0)[0]
+        free = rng.permutation(np.arange(-2, doc_cap + 2)).astype(np.int32)
+        take = min(len(doc_rows), len(free))
+        pos[doc_rows[:take]] = free[:take]
+        sid[doc_rows[take:]] = -1
+        k = wl.randn_bf16((n, H, d), 300 + call, DEV)
+        v = wl.randn_bf16((n, H, d), 400 + call, DEV)
+        m.kv_append(layer, k, v, torch.from_numpy(sid).to(DEV), torch.from_numpy(pos).to(DEV))
+        R.append(bf16_bits(k), bf16_bits(v), sid, pos)
+    torch.cuda.synchronize()
+    ln = layer.len.cpu().numpy()
+    ks, vs = bf16_bits(layer.k_suf), bf16_bits(layer.v_suf)
+    tag_s, tag_p = layer.sid.cpu().numpy(), layer.pos.cpu().numpy()
+    for s in range(1, P_max + 1):
+        assert ln[s - 1] == R.length(s)
+        seg = R.seg[s]
+        if seg:
+            assert np.array_equal(ks[s - 1, :, :len(seg), :], np.stack([x[0] for x in seg], 1))
+            assert np.array_equal(vs[s - 1, :, :len(seg), :], np.stack([x[1] for x in seg], 1))
+            assert np.array_equal(tag_s[s - 1, :len(seg)], [x[2] for x in seg])
+            assert np.array_equal(tag_p[s - 1, :len(seg)], [x[3] for x in seg])
+    kd, vd = bf16_bits(layer.k_doc), bf16_bits(layer.v_doc)
+    for p_, (kk, vv) in R.doc.items():
+        assert np.array_equal(kd[:, p_, :], kk) and np.array_equal(vd[:, p_, :], vv)
+    flags = {"segment_overflow": m.PP_DEV_SEGMENT_OVERFLOW,
+             "doc_out_of_range": m.PP_DEV_DOC_OUT_OF_RANGE, "bad_stream": m.PP_DEV_BAD_STREAM}
+    expect = 0
+    for f in R.flags:
+        expect |= flags[f]
+    assert expect & m.PP_DEV_SEGMENT_OVERFLOW
+    assert m.device_status(layer) == expect
+
+
 def test_append_many_rows_per_stream_keeps_call_order():
     m = gu.pp()
     H, d, P_max, S_cap = 2, 128, 4, 300
