@@ -25,6 +25,26 @@ def declared_functions():
     return sorted(set(re.findall(r"\b(pp_[a-z_0-9]+)\s*\(", src)))
 
 
+def header_struct_fields(name):
+    """Field names, in order, of `typedef struct name {...} name;` in the header."""
+    src = open(os.path.join(ROOT, "include", "ppattn.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    body = re.search(r"typedef struct " + name + r"\s*\{(.*?)\}\s*" + name + ";", src, re.S).group(1)
+    fields = []
+    for decl in body.split(";"):
+        if decl.strip():
+            _type, names = decl.strip().split(None, 1)
+            fields += [x.strip().lstrip("*").strip() for x in names.split(",")]
+    return fields
+
+
+def test_ctypes_structs_match_the_header(pp):
+    """The binding's layer descriptor and options mirror the C structs field by
+    field (a reordered or missing field would silently shift every later one)."""
+    assert [f for f, _ in pp.LayerStruct._fields_] == header_struct_fields("pp_kv_layer")
+    assert [f for f, _ in pp.Options._fields_] == header_struct_fields("pp_options")
+
+
 def test_header_declares_the_three_calls():
     names = declared_functions()
     for n in ("pp_kv_append", "pp_decode_attn", "pp_prefill_attn"):
