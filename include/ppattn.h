@@ -178,8 +178,11 @@ pp_status pp_kv_append(const pp_kv_layer *layer, const uint16_t *k, const uint16
                        const int16_t *sid, const int32_t *pos, int32_t n, void *stream);
 
 /*
- * Workspace bytes pp_decode_attn needs for P query rows (fp32 partial
- * results of the split document pass; 0 when doc_len is 0).  The split
+ * Workspace bytes pp_decode_attn and pp_decode_step need for P query rows
+ * (fp32 partial results of the split document pass; one int per row for
+ * the stream lengths of a step whose append runs inside that pass; arrival
+ * counters and fp32 partials for suffix items cut between warps; 0 when
+ * doc_len is 0).  The split
  * plan depends on the SM count of the CURRENT device: query with the device
  * that will run the call.  Returns 0 on bad arguments or without a device.
  */
