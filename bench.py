@@ -767,6 +767,9 @@ def main():
     ap.add_argument("--separate-append", action="store_true",
                     help="decode: pp_kv_append + pp_decode_attn per layer instead of "
                          "pp_decode_step (append inside the document pass), for comparison")
+    ap.add_argument("--suffix-slices", type=int, default=0, choices=[0, 1, 2],
+                    help="decode: how the suffix pass's warps share the work "
+                         "(pp_options.suffix_slices; 0 = automatic)")
     ap.add_argument("--mode", default="decode",
                     choices=["decode", "prefill", "ablation", "siblingscan", "sweep", "docprefill",
                              "longanswer"],
@@ -800,6 +803,8 @@ def main():
     nl = args.layers or wl.CONFIGS[args.workload]["layers"]
     step = DecodeStep(args.workload, nl, dev)
     step.fused = not args.separate_append
+    if args.suffix_slices:
+        step.opts = [step.pp.Options(suffix_slices=args.suffix_slices) for _ in range(nl)]
     W = step.W
     step.capture()
 
@@ -891,6 +896,8 @@ def main():
                              if nl == 32 else "per-layer document KV exceeds L2",
                        "append": "inside the document pass (pp_decode_step)" if step.fused
                                  else "separate kernels (pp_kv_append)",
+                       "suffix_slices": {0: "automatic", 1: "equal item counts",
+                                         2: "balanced by work"}[args.suffix_slices],
                        "parallelism": f"replicas x{world}"},
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},

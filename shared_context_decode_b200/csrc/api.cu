@@ -195,7 +195,8 @@ pp_status attend(const pp_kv_layer* L, int32_t doc_len, const uint16_t* q, const
   const bool want = slices == 2 ||
                     (slices == 0 && ((int64_t)rows * L->H < 2LL * sms * pp::kSuffixWarps ||
                                      L->S_cap > 32 * 16));
-  const bool balance = want && read_once && has_doc && !other_doc && rows <= pp::kBalanceRows;
+  const bool balance = want && read_once && has_doc && !other_doc && rows <= pp::kBalanceRows &&
+                       (int64_t)rows * L->H < (1LL << 31);
   if (balance) {
     split.cnt = reinterpret_cast<int32_t*>(wsb + w.split_cnt);
     split.o = reinterpret_cast<float*>(wsb + w.split_o);

@@ -302,7 +302,7 @@ __global__ void __launch_bounds__(SufCfg<D, BAL>::WARPS * 32) suffix_merge(const
       rec.n = 0;
       rec.raw = s;
       if constexpr (balanced) {  // this warp's units of the item, as keys
-        const int64_t S = (item / p.rows) * Ctot + pre[r];
+        const int64_t S = (int64_t)((int)item / p.rows) * Ctot + pre[r];  // items < 2^31
         const int64_t U = pre[r + 1] - pre[r];
         rec.set_range((int)((u_lo > S ? u_lo - S : 0) * C::CK),
                       (int)((u_hi < S + U ? u_hi - S : U) * C::CK));
@@ -546,10 +546,13 @@ __global__ void __launch_bounds__(SufCfg<D, BAL>::WARPS * 32) suffix_merge(const
       if constexpr (balanced) {
         // an item cut by slice boundaries: publish this warp's partial; the
         // last of its warps to arrive folds the others in and finishes it
+        // (only items longer than kSnapUnits can be cut: the others skip
+        // the 64-bit divisions of warp_of)
         const int64_t S = (int64_t)h * Ctot + pre[r];
         const int U = pre[r + 1] - pre[r];
-        const int64_t wf = warp_of(S), wl = warp_of(S + U - 1);
-        if (U > kSnapUnits && wf != wl) {
+        const int64_t wf = U > kSnapUnits ? warp_of(S) : 0;
+        const int64_t wl = U > kSnapUnits ? warp_of(S + U - 1) : 0;
+        if (wf != wl) {
           // partial slot: 2 w for the warp's first item, 2 w + 1 for its last
           const int64_t slot = 2 * gw + (item == i_first ? 0 : 1);
 #pragma unroll
