@@ -105,7 +105,10 @@ class ClockSampler:
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv")
+        # raw samples: $PP_CLOCKS_DIR if set, else the system temporary directory
+        import tempfile
+        d = os.environ.get("PP_CLOCKS_DIR") or tempfile.gettempdir()
+        self.path = os.path.join(d, f"pp_clocks_rank{gpu_index}.csv")
         self.t_start = self.t_end = None
 
     def __enter__(self):
