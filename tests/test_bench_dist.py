@@ -86,3 +86,19 @@ def test_reference_arm_line_on_rank_zero(capsys):
                            "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
     assert line["config"]["workload"] == "tiny"
+
+
+def test_profile_traffic_only_while_the_sources_match(tmp_path):
+    """roofline.traffic comes from a committed ncu summary only while the
+    kernel's sources hash to the value recorded with it."""
+    sys.path.insert(0, ROOT)
+    import bench
+    good = tmp_path / "good.md"
+    good.write_text(f"- sources sha256: `{bench.kernel_source_hash()}`\n"
+                    "- dram bytes per launch (read + write): 123456\n")
+    assert bench.profile_traffic(str(good)) == 123456.0
+    stale = tmp_path / "stale.md"
+    stale.write_text("- sources sha256: `" + "0" * 64 + "`\n"
+                     "- dram bytes per launch (read + write): 123456\n")
+    assert bench.profile_traffic(str(stale)) is None
+    assert bench.profile_traffic(str(tmp_path / "absent.md")) is None
