@@ -54,7 +54,7 @@ typedef enum pp_status {
     PP_ERR_UNSUPPORTED = 2,     /* d not in {64,128}, P > P_max, P > 32767    */
     PP_ERR_CAPACITY = 3,        /* doc_len > doc_cap, workspace too small     */
     PP_ERR_CUDA = 4,            /* a CUDA launch or driver call failed        */
-    PP_ERR_DEVICE_TIMEOUT = 5   /* reserved for callers mapping PP_DEV_TIMEOUT */
+    PP_ERR_DEVICE_TIMEOUT = 5   /* pp_get_device_status: PP_DEV_TIMEOUT is set */
 } pp_status;
 
 /* Bits of the per-layer device status word (sticky; cleared by pp_kv_reset). */
@@ -254,6 +254,11 @@ pp_status pp_decode_step(const pp_kv_layer *layer, int32_t doc_len, const uint16
  *     stream capture.
  *   - Every call shares the one scratch array: calls whose kernels overlap on
  *     the GPU (different streams, unordered) corrupt each other's results.
+ *   - The looked-up address is kept for the life of the process.  A
+ *     cudaDeviceReset frees the array behind it, so this call must not be
+ *     used on a device after that device has been reset.
+ *   - Invalid arguments get the same status as from pp_decode_attn
+ *     (PP_ERR_INVALID_ARG, PP_ERR_UNSUPPORTED), checked before the size.
  */
 #define PP_NOALLOC_SCRATCH_BYTES (32u << 20)
 pp_status pp_decode_attn_noalloc(const pp_kv_layer *layer, int32_t doc_len, const uint16_t *q,
@@ -346,7 +351,11 @@ pp_status pp_debug_split_plan_causal(int32_t doc_len, int32_t H, int32_t ctas, i
  */
 pp_status pp_debug_exp2(const float *x, float *y_poly, float *y_hw, int32_t n, void *stream);
 
-/* Copy the layer's device status word to *h_status (synchronises stream). */
+/* Copy the layer's device status word to *h_status (synchronises stream).
+ * Returns PP_ERR_DEVICE_TIMEOUT when the word has PP_DEV_TIMEOUT set (a
+ * bounded in-kernel wait gave up: that call's outputs are not valid), with
+ * *h_status written all the same; PP_OK otherwise, whatever the other bits
+ * (they report dropped or rejected rows, not failed launches). */
 pp_status pp_get_device_status(const pp_kv_layer *layer, int32_t *h_status, void *stream);
 
 #ifdef __cplusplus

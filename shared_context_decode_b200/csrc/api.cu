@@ -33,6 +33,9 @@ int sm_count() {
   return n;
 }
 
+}  // namespace
+
+namespace pp {
 pp_status check_layer(const pp_kv_layer* L) {
   if (!L) return PP_ERR_INVALID_ARG;
   if (L->d != 64 && L->d != 128) return PP_ERR_UNSUPPORTED;
@@ -47,6 +50,10 @@ pp_status check_layer(const pp_kv_layer* L) {
     return PP_ERR_INVALID_ARG;
   return PP_OK;
 }
+}  // namespace pp
+
+namespace {
+using pp::check_layer;
 
 pp_status from_cuda(cudaError_t e) { return e == cudaSuccess ? PP_OK : PP_ERR_CUDA; }
 
@@ -406,7 +413,8 @@ PP_API pp_status pp_get_device_status(const pp_kv_layer* layer, int32_t* h_statu
   if (cudaMemcpyAsync(h_status, layer->status, sizeof(int32_t), cudaMemcpyDeviceToHost, st) !=
       cudaSuccess)
     return PP_ERR_CUDA;
-  return from_cuda(cudaStreamSynchronize(st));
+  if ((s = from_cuda(cudaStreamSynchronize(st))) != PP_OK) return s;
+  return (*h_status & PP_DEV_TIMEOUT) ? PP_ERR_DEVICE_TIMEOUT : PP_OK;
 }
 
 }  // extern "C"

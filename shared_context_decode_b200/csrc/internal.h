@@ -21,6 +21,10 @@ bool make_tmap_bf16_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d
 
 struct AppendJob;
 
+// Host validation of a layer descriptor (the checks every entry point runs
+// first): PP_OK, PP_ERR_INVALID_ARG or PP_ERR_UNSUPPORTED.
+pp_status check_layer(const pp_kv_layer* L);
+
 // streams_only: rows of stream 0 are skipped instead of written to the
 // document block (a decode step carries no document rows).
 cudaError_t launch_kv_append(const pp_kv_layer& L, const uint16_t* k, const uint16_t* v,

@@ -14,6 +14,9 @@
 // the first call on each device looks the address up (cudaGetSymbolAddress,
 // with that device current) and caches it.
 //
+// The address is kept for the life of the process; a cudaDeviceReset frees
+// the array behind it, so the entry point is not for use after a reset.
+//
 // All calls share the one array, on every stream.  Nothing in it needs to
 // start at zero (each call writes every partial it later reads), but calls
 // whose kernels overlap on the GPU overwrite each other's partials: the caller
@@ -54,7 +57,10 @@ extern "C" __attribute__((visibility("default"))) pp_status pp_decode_attn_noall
     const pp_kv_layer* layer, int32_t doc_len, const uint16_t* q, const int16_t* q_sid,
     const int32_t* q_pos, int32_t P, float scale, uint16_t* o, float* lse, const pp_options* opt,
     void* stream) {
-  if (!layer) return PP_ERR_INVALID_ARG;
+  // The argument errors pp_decode_attn reports come first, with its codes.
+  const pp_status v = pp::check_layer(layer);
+  if (v != PP_OK) return v;
+  if (P > layer->P_max) return PP_ERR_UNSUPPORTED;
   // Too much for the fixed scratch: refuse before touching anything.
   // (0 means nothing is needed, or arguments pp_decode_attn will reject.)
   if (pp_decode_workspace_bytes(P, layer->H, layer->d, doc_len, opt) > PP_NOALLOC_SCRATCH_BYTES)

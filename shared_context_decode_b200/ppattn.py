@@ -383,10 +383,19 @@ def debug_exp2(x: torch.Tensor):
 
 
 def device_status(layer: KVLayer) -> int:
+    """The layer's device status word (PP_DEV_* bits).  A word with
+    PP_DEV_TIMEOUT set is returned too (the call reports it as
+    PP_ERR_DEVICE_TIMEOUT; device_status_code gives that code)."""
+    return device_status_code(layer)[1]
+
+
+def device_status_code(layer: KVLayer):
+    """(pp_status of pp_get_device_status, status word)."""
     out = _i32(0)
-    _check(_dev_status(layer.ref, ctypes.byref(out), _stream(layer.device)),
-           "pp_get_device_status")
-    return int(out.value)
+    rc = int(_dev_status(layer.ref, ctypes.byref(out), _stream(layer.device)))
+    if rc not in (PP_OK, PP_ERR_DEVICE_TIMEOUT):
+        _check(rc, "pp_get_device_status")
+    return rc, int(out.value)
 
 
 def split_plan(rows: int, H: int, doc_len: int, ctas: int, causal: bool = False):

@@ -126,6 +126,14 @@ def test_host_validation_codes(pp):
     # visibility
     assert pp._visibility(ctypes.byref(L), 5, 0x1000, 0x2000, -1, 0x3000, None, None) == \
         pp.PP_ERR_INVALID_ARG
+    # no-alloc decode: argument errors come first, with pp_decode_attn's codes
+    # (a P far above the layer's streams is not reported as a size problem)
+    def noalloc(lay, P=4):
+        return pp._decode_noalloc(ctypes.byref(lay), 10, 0x90000, 0xA0000, 0xB0000, P, 0.1,
+                                  0xC0000, None, None, None)
+    assert noalloc(L, P=100000) == pp.PP_ERR_UNSUPPORTED
+    assert noalloc(fake_layer(pp, d=96)) == pp.PP_ERR_UNSUPPORTED
+    assert noalloc(fake_layer(pp, len=0)) == pp.PP_ERR_INVALID_ARG
 
 
 def test_workspace_sizes_with_explicit_split(pp):

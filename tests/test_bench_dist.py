@@ -102,3 +102,28 @@ def test_profile_traffic_only_while_the_sources_match(tmp_path):
                      "- dram bytes per launch (read + write): 123456\n")
     assert bench.profile_traffic(str(stale)) is None
     assert bench.profile_traffic(str(tmp_path / "absent.md")) is None
+
+
+def test_doc_roofline_uses_the_burst_peak_and_reports_the_stricter_gate():
+    """The document pass's roofline: roof time = the slower of the bytes at
+    the measured copy rate and the FLOPs at the burst bf16 rate; frac = roof
+    time / measured time.  The nominal figures give the stricter gate."""
+    sys.path.insert(0, ROOT)
+    import bench
+    from shared_context_decode_b200 import workloads as wl
+    W = wl.make_decode("doc16k_p256", device="cpu")
+    peaks = dict(hbm=6548.0, bf16=1629.0, bf16_sustained=1390.0, source="measured")
+    r = bench.doc_roofline(W, {"doc": 0.0725, "suffix": 0.0594}, peaks, None)
+    b, f = 2 * 16384 * 32 * 128 * 2, 4 * 256 * 16384 * 128 * 32
+    t_roof = max(b / 6548e9, f / 1629e12)
+    assert r["bound"] == "tensor" and r["peak"] == 1629.0
+    assert r["frac"] == pytest.approx(t_roof / 72.5e-6)
+    assert r["frac"] == pytest.approx(r["achieved"] / r["peak"])
+    assert r["frac_spec"] == pytest.approx(max(b / 8e12, f / 2.25e15) / 72.5e-6)
+    assert r["frac_gate"] == pytest.approx(min(r["frac"], r["frac_spec"]))
+    assert r["frac_sustained"] > r["frac"]
+    # a memory-bound workload (64 streams) is bound by HBM
+    W2 = wl.make_decode("doc8k_p64", device="cpu")
+    r2 = bench.doc_roofline(W2, {"doc": 0.030, "suffix": 0.010}, peaks, None)
+    assert r2["bound"] == "hbm" and r2["unit"] == "GB/s"
+    assert r2["frac"] == pytest.approx((2 * 8192 * 32 * 128 * 2 / 6548e9) / 30e-6)

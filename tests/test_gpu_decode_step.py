@@ -79,13 +79,14 @@ def test_step_equals_append_then_attend(case):
     gu.compare(o, lse, ref_o, ref_lse, case)
 
 
-def test_full_size_step_sampled():
-    W = wl.make_decode("doc16k_p256", layers=1, device=DEV)
+@pytest.mark.parametrize("name", ["doc8k_p64", "doc16k_p256"])
+def test_full_size_step_whole_layer(name):
+    """The fused step at full size: every row and head of one layer."""
+    W = wl.make_decode(name, layers=1, device=DEV)
     L = W.layer(0)
     o, lse, _ = step_vs_separate(W, L, L.new_k, L.new_v, L.q, L.q_sid, L.q_pos)
-    rows = np.sort(np.random.default_rng(2).choice(W.P, size=8, replace=False))
-    ref_o, ref_lse, _ = gu.oracle_decode(W, L, rows)
-    gu.compare(o[rows], lse[rows], ref_o, ref_lse, "doc16k_p256 step")
+    ref_o, ref_lse, _ = gu.oracle_decode(W, L)
+    gu.compare(o, lse, ref_o, ref_lse, f"{name} step")
 
 
 def test_duplicates_overflow_and_bad_rows_bit_exact():

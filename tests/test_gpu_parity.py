@@ -3,14 +3,16 @@
 Small cases are compared in full and span several document tiles, both M
 tiles of a row group, two row groups, ragged tails and forced split counts
 that make CTAs cross head boundaries; the named full-size workloads are
-compared on sampled rows (all heads, all d) in the launch configuration the
-bench uses.
+compared on whole layers (every row, head and dimension) in the launch
+configuration the bench uses.
 """
 import numpy as np
 import pytest
 import torch
 
+import oracle
 from shared_context_decode_b200 import workloads as wl
+from tests import flat
 from tests import gpu_util as gu
 
 pytestmark = pytest.mark.gpu
@@ -41,6 +43,27 @@ def test_ragged_two_mtiles_split_variants(splits):
                        device=DEV)
     opt = gu.pp().Options(splits=splits) if splits else None
     decode_case(W, opt=opt)
+
+
+@pytest.mark.parametrize("P", [64, 128])
+@pytest.mark.parametrize("splits", [1, 3, 7, 20, 32])
+def test_single_mtile_tile_parity_split(P, splits):
+    """Row groups with one M tile: the two softmax warpgroups take alternate
+    key tiles of it and combine at the end of each segment, including
+    segments of one tile (the second warpgroup then has none) and of odd
+    length; 8 key tiles with a 104-key tail, 4 heads."""
+    W = wl.make_decode(layers=1, H=4, d=128, N=1000, P=P, q=(1, 20), a=(0, 10), seed=31,
+                       device=DEV)
+    decode_case(W, opt=gu.pp().Options(splits=splits))
+
+
+@pytest.mark.parametrize("splits", [1, 4, 9, 25, 33])
+def test_mixed_mtile_modes_across_segments(splits):
+    """P = 300: the first row group has two M tiles, the second one (44 rows)
+    only one, so CTAs cross between the two modes of the document pass."""
+    W = wl.make_decode(layers=1, H=3, d=128, N=1000, P=300, q=(1, 9), a=(0, 4), seed=32,
+                       device=DEV)
+    decode_case(W, opt=gu.pp().Options(splits=splits))
 
 
 def test_two_row_groups():
@@ -85,6 +108,27 @@ def test_inactive_rows_are_zero():
     assert torch.all(torch.isinf(lse[torch.from_numpy(~active).to(DEV)]))
 
 
+@pytest.mark.parametrize("P,H,d,a,active_every", [(300, 16, 128, (0, 40), 3), (5000, 1, 64, (0, 20), 0),
+                                                  (257, 14, 128, (0, 63), 0)])
+def test_equal_item_counts_longest_first(P, H, d, a, active_every):
+    """The suffix pass with equal item counts per warp: each CTA sorts the
+    rows by work and deals the items longest first.  Inactive rows (no work,
+    sorted last), a row count above the sorted limit (contiguous items
+    instead) and a ragged head count."""
+    m = gu.pp()
+    W = wl.make_decode(layers=1, H=H, d=d, N=300, P=P, q=(1, 20), a=a, seed=33, device=DEV)
+    active = (np.arange(P) % active_every != 1) if active_every else None
+    L = W.layer(0, active=active)
+    layer = gu.load_decode(W, L, DEV)
+    lse = torch.empty((W.P, W.H), dtype=torch.float32, device=DEV)
+    o = m.decode_attn(layer, W.N, L.q, L.q_sid, L.q_pos, W.scale, lse=lse,
+                      opt=m.Options(suffix_slices=1))
+    torch.cuda.synchronize()
+    assert m.device_status(layer) == 0
+    o_ref, lse_ref, _ = gu.oracle_decode(W, L)
+    gu.compare(o, lse, o_ref, lse_ref, "longest first")
+
+
 def test_doc_pass_stays_in_segment_when_other_streams_longer():
     # Streams with very different suffix lengths; the mask must not leak.
     W = wl.make_decode(layers=1, H=2, d=128, N=400, P=9, q=(1, 60), a=(0, 60), seed=8, device=DEV)
@@ -92,12 +136,12 @@ def test_doc_pass_stays_in_segment_when_other_streams_longer():
 
 
 @pytest.mark.parametrize("name", ["doc8k_p64", "doc16k_p256"])
-def test_full_size_sampled(name):
+def test_full_size_whole_layers(name):
+    """Every row, head and output dimension of the first and the last layer
+    of the full-size workloads, in the bench's launch configuration."""
     W = wl.make_decode(name, device=DEV)
-    rng = np.random.default_rng(0)
-    rows = np.sort(rng.choice(W.P, size=min(W.P, 12), replace=False))
     for l in (0, W.layers - 1):
-        decode_case(W, l=l, rows=rows)
+        decode_case(W, l=l)
 
 
 @pytest.mark.parametrize("P,H,q,a", [(3, 2, (10, 20), (1500, 2500)), (40, 2, (1, 30), (0, 600)),
@@ -164,7 +208,10 @@ def test_prefill_small_full():
     gu.compare(o, lse, o_ref, lse_ref, "prefill small")
 
 
-def test_prefill_full_size_sampled():
+def test_prefill_full_size():
+    """Question prefill at full size (8260 rows, 33 row groups): every row of
+    the first 256-row group, of a middle group and of the ragged last group
+    on all heads, and every row of the call on the first and the last head."""
     m = gu.pp()
     W = wl.make_prefill("prefill_doc12k_p256", device=DEV)
     L = W.layer(0)
@@ -173,7 +220,14 @@ def test_prefill_full_size_sampled():
     o = m.prefill_attn(layer, W.N, L.q, L.sid, L.pos, W.scale, lse=lse)
     torch.cuda.synchronize()
     assert m.device_status(layer) == 0
-    rng = np.random.default_rng(1)
-    rows = np.sort(rng.choice(W.R, size=16, replace=False))
+    G = -(-W.R // 256)
+    rows = np.concatenate([np.arange(0, 256), np.arange(256 * (G // 2), 256 * (G // 2 + 1)),
+                           np.arange(256 * (G - 1), W.R)])
     o_ref, lse_ref, _ = gu.oracle_prefill(W, L, rows)
-    gu.compare(o[rows], lse[rows], o_ref, lse_ref, "prefill full")
+    gu.compare(o[rows], lse[rows], o_ref, lse_ref, "prefill full, three row groups")
+    heads = [0, W.H - 1]
+    k, v, ks, kp = flat.prefill_slots(L, W.N)
+    q, qs, qp = flat.prefill_queries(L)
+    o_ref, lse_ref, _ = oracle.masked_attention(q[:, heads], qs, qp, k[:, heads], v[:, heads],
+                                                ks, kp, W.scale)
+    gu.compare(o[:, heads], lse[:, heads], o_ref, lse_ref, "prefill full, every row")

@@ -25,13 +25,14 @@ def test_injected_timeout_reports_status_and_recovers():
     opt = m.Options(debug_inject_timeout=1, wait_limit_log2=22)   # ~2^22 cycles per wait
     m.decode_attn(layer, W.N, L.q, L.q_sid, L.q_pos, W.scale, opt=opt)
     torch.cuda.synchronize()
-    assert m.device_status(layer) & m.PP_DEV_TIMEOUT
+    rc, word = m.device_status_code(layer)
+    assert word & m.PP_DEV_TIMEOUT and rc == m.PP_ERR_DEVICE_TIMEOUT
     # the context is intact: a normal call on the same layer is correct
     layer.status.zero_()
     lse = torch.empty((W.P, W.H), dtype=torch.float32, device=DEV)
     o = m.decode_attn(layer, W.N, L.q, L.q_sid, L.q_pos, W.scale, lse=lse)
     torch.cuda.synchronize()
-    assert m.device_status(layer) == 0
+    assert m.device_status_code(layer) == (m.PP_OK, 0)
     o_ref, lse_ref, _ = gu.oracle_decode(W, L)
     gu.compare(o, lse, o_ref, lse_ref, "after timeout")
 

@@ -3,9 +3,10 @@ device memory (for example a plugin inside a host application that owns all
 device memory and offers it no allocator, or a serving loop that forbids
 cudaMalloc after start-up because it can synchronise the device).
 
-It must give the same results as pp_decode_attn with a caller-allocated
-workspace, call after call (its built-in scratch is reused), and it must
-refuse work that needs more scratch than it has.  This file is collected
+It runs the same kernels on the same split as pp_decode_attn with a
+caller-allocated workspace, so it must give the same bits, call after call
+(its built-in scratch is reused); it must refuse work that needs more
+scratch than it has, and report argument errors as pp_decode_attn does.  This file is collected
 last, so a run that stops at the first failure has run everything else."""
 import numpy as np
 import pytest
@@ -29,12 +30,9 @@ def _compare_to_workspace_call(W, l=0):
     m.decode_attn_noalloc(layer, W.N, L.q, L.q_sid, L.q_pos, W.scale, o=o, lse=lse)
     torch.cuda.synchronize()
     assert m.device_status(layer) == 0
-    err = (o.float() - o_ref.float()).abs()
     assert torch.isfinite(o.float()).all()
-    assert err.max().item() <= gu.O_MAX and err.mean().item() <= gu.O_MEAN
-    fin = torch.isfinite(lse_ref)
-    assert torch.equal(fin, torch.isfinite(lse))
-    assert (lse[fin] - lse_ref[fin]).abs().max().item() <= gu.LSE_MAX
+    assert torch.equal(o.view(torch.int16), o_ref.view(torch.int16))
+    assert torch.equal(lse, lse_ref)
 
 
 def test_noalloc_matches_workspace_entry_point_two_calls_in_a_row():
@@ -63,3 +61,9 @@ def test_noalloc_rejects_work_beyond_its_scratch():
     assert e.value.status == m.PP_ERR_CAPACITY
     torch.cuda.synchronize()
     assert torch.all(o == 7.0)               # nothing was launched
+    # more rows than the layer has streams: the argument error comes first,
+    # with pp_decode_attn's code, although the size is also too large
+    small = m.KVLayer(H, d, N, 8, 8, DEV)
+    with pytest.raises(m.PPError) as e:
+        m.decode_attn_noalloc(small, N, q, sid, pos, 0.1, o=o)
+    assert e.value.status == m.PP_ERR_UNSUPPORTED
