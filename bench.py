@@ -335,6 +335,41 @@ class PrefillStep:
         return self.layers * 4
 
 
+def eager_e2e(step, host_in, host_out, names, steps: int, world: int, dev):
+    """The decode step end to end with no graph: for each layer, copy its
+    inputs from pinned host memory, call the C ABI (pp_decode_step, or the
+    step's configured calls), copy o back, all on the current stream.
+    Returns the throughput, the device time per step and the host time spent
+    issuing one layer (copies + C-ABI call), the per-call host cost a caller
+    that does not capture a graph pays."""
+    cur = torch.cuda.current_stream(dev)
+
+    def one():
+        step.len_all.copy_(step.len0)
+        for l in range(step.layers):
+            x = step.inp[l]
+            for n in names:
+                x[n].copy_(host_in[l][n], non_blocking=True)
+            step.layer_call(l, None if step.opts is None else step.opts[l])
+            host_out[l].copy_(x["o"], non_blocking=True)
+
+    one()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    host_s = 0.0
+    e0.record(cur)
+    for _ in range(steps):
+        t0 = time.perf_counter()
+        one()
+        host_s += time.perf_counter() - t0
+    e1.record(cur)
+    torch.cuda.synchronize()
+    value, ms = aggregate(step.W.P, e0.elapsed_time(e1) / steps, world, dev)
+    return {"value": value, "unit": UNIT, "ms_per_step": ms,
+            "host_us_per_layer_call": host_s / steps / step.layers * 1e6,
+            "form": "eager: per layer copies in, one C-ABI call, o copied out"}
+
+
 def timed_replays(step, steps: int, warmup: int, world: int, local: int):
     for _ in range(warmup):
         step.replay()
@@ -946,6 +981,12 @@ def main():
         if not torch.equal(host_out[l], step.inp[l]["o"].cpu()):
             raise RuntimeError(f"end-to-end output of layer {l} differs from the device step")
 
+    # ---- end to end without a graph: per layer, the host->device copies of
+    # its inputs, the C-ABI call and the copy of o back, issued eagerly on
+    # one stream; the wall time of the issuing loop alone gives the host
+    # cost per C-ABI call
+    eager = eager_e2e(step, host_in, host_out, names, max(3, args.steps // 10), world, dev)
+
     # ---- roofline of the dominant kernel (document pass), live CUDA events
     durs = measure_doc_pass(step, args.roofline_reps)
     roof = doc_roofline(W, durs, load_peaks(), profile_traffic(doc_profile(args.workload)))
@@ -973,7 +1014,9 @@ def main():
                                          2: "balanced by work"}[args.suffix_slices],
                        "parallelism": f"replicas x{world}"},
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
-                    "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+                    "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+                    "form": "one CUDA graph per step (copies overlapped on three streams)",
+                    "eager": eager},
             "gpu_launches": step.kernels_per_step() * args.steps,
             "roofline": roof,
             "cpu_baseline": cpu,

@@ -5,6 +5,8 @@
 //   decode / prefill:  [document pass] -> suffix pass with the merge fused
 // Nothing here allocates device memory or synchronises (except
 // pp_get_device_status), so the calls can be captured in a CUDA graph.
+#include <nvtx3/nvToolsExt.h>
+
 #include <algorithm>
 #include <atomic>
 
@@ -56,6 +58,16 @@ namespace {
 using pp::check_layer;
 
 pp_status from_cuda(cudaError_t e) { return e == cudaSuccess ? PP_OK : PP_ERR_CUDA; }
+
+// A named NVTX range around an entry point, so a profiler's timeline shows
+// each C-ABI call (header-only NVTX: without an attached tool a push/pop is
+// a check of a null function pointer).
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 // The document split: see pp::SplitPlan.  `ctas` = slots to spread it over;
 // `causal`: a document prefill (rows = document tokens, triangular units).
@@ -293,6 +305,7 @@ PP_API const char* pp_status_str(int32_t status) {
 PP_API int32_t pp_abi_version(void) { return PP_ABI_VERSION; }
 
 PP_API pp_status pp_kv_reset(const pp_kv_layer* layer, void* stream) {
+  NvtxRange nvtx_range("pp_kv_reset");
   pp_status s = check_layer(layer);
   if (s != PP_OK) return s;
   return from_cuda(pp::launch_kv_reset(*layer, static_cast<cudaStream_t>(stream)));
@@ -300,6 +313,7 @@ PP_API pp_status pp_kv_reset(const pp_kv_layer* layer, void* stream) {
 
 PP_API pp_status pp_kv_reset_streams(const pp_kv_layer* layer, const int16_t* sid, int32_t n,
                                      void* stream) {
+  NvtxRange nvtx_range("pp_kv_reset_streams");
   pp_status s = check_layer(layer);
   if (s != PP_OK) return s;
   if (n < 0) return PP_ERR_INVALID_ARG;
@@ -311,6 +325,7 @@ PP_API pp_status pp_kv_reset_streams(const pp_kv_layer* layer, const int16_t* si
 
 PP_API pp_status pp_kv_append(const pp_kv_layer* layer, const uint16_t* k, const uint16_t* v,
                        const int16_t* sid, const int32_t* pos, int32_t n, void* stream) {
+  NvtxRange nvtx_range("pp_kv_append");
   pp_status s = check_layer(layer);
   if (s != PP_OK) return s;
   if (n < 0) return PP_ERR_INVALID_ARG;
@@ -335,6 +350,7 @@ PP_API pp_status pp_decode_attn(const pp_kv_layer* layer, int32_t doc_len, const
                          const int16_t* q_sid, const int32_t* q_pos, int32_t P, float scale,
                          uint16_t* o, float* lse, void* ws, size_t ws_bytes, const pp_options* opt,
                          void* stream) {
+  NvtxRange nvtx_range("pp_decode_attn");
   if (layer && P > layer->P_max) return PP_ERR_UNSUPPORTED;
   return attend(layer, doc_len, q, q_sid, q_pos, P, scale, o, lse, ws, ws_bytes, opt, stream,
                 false, true);
@@ -345,6 +361,7 @@ PP_API pp_status pp_decode_step(const pp_kv_layer* layer, int32_t doc_len, const
                                 const int32_t* q_pos, int32_t P, float scale, uint16_t* o,
                                 float* lse, void* ws, size_t ws_bytes, const pp_options* opt,
                                 void* stream) {
+  NvtxRange nvtx_range("pp_decode_step");
   if (layer && P > layer->P_max) return PP_ERR_UNSUPPORTED;
   if (P > 0 && (!k || !v || !aligned(k, 16) || !aligned(v, 16))) return PP_ERR_INVALID_ARG;
   return attend(layer, doc_len, q, q_sid, q_pos, P, scale, o, lse, ws, ws_bytes, opt, stream,
@@ -355,6 +372,7 @@ PP_API pp_status pp_prefill_attn(const pp_kv_layer* layer, int32_t doc_len, cons
                           const int16_t* q_sid, const int32_t* q_pos, int32_t R, float scale,
                           uint16_t* o, float* lse, void* ws, size_t ws_bytes,
                           const pp_options* opt, void* stream) {
+  NvtxRange nvtx_range("pp_prefill_attn");
   return attend(layer, doc_len, q, q_sid, q_pos, R, scale, o, lse, ws, ws_bytes, opt, stream);
 }
 
@@ -366,6 +384,7 @@ PP_API size_t pp_doc_prefill_workspace_bytes(int32_t H, int32_t d, int32_t doc_l
 PP_API pp_status pp_doc_prefill_attn(const pp_kv_layer* layer, int32_t doc_len, const uint16_t* q,
                                      float scale, uint16_t* o, float* lse, void* ws,
                                      size_t ws_bytes, const pp_options* opt, void* stream) {
+  NvtxRange nvtx_range("pp_doc_prefill_attn");
   return attend(layer, doc_len, q, nullptr, nullptr, doc_len, scale, o, lse, ws, ws_bytes, opt,
                 stream, true);
 }
@@ -406,6 +425,7 @@ PP_API pp_status pp_debug_exp2(const float* x, float* y_poly, float* y_hw, int32
 }
 
 PP_API pp_status pp_get_device_status(const pp_kv_layer* layer, int32_t* h_status, void* stream) {
+  NvtxRange nvtx_range("pp_get_device_status");
   pp_status s = check_layer(layer);
   if (s != PP_OK) return s;
   if (!h_status) return PP_ERR_INVALID_ARG;

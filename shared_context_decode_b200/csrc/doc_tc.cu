@@ -492,16 +492,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int e = 0; e < 32; ++e)
               if (c * 32 + e >= kvalid) r[c][e] = __float_as_uint(-INFINITY);
         }
-        // partial row maximum: 8 independent chains of 3-input max
-        float mc[8];
+        float mc[16];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) mc[k] = -INFINITY;
+        for (int k = 0; k < 16; ++k) mc[k] = -INFINITY;
 #pragma unroll
-        for (int i = 0; i < HB; i += 2)
-          mc[(i >> 1) & 7] = fmax3(mc[(i >> 1) & 7], __uint_as_float(r[i >> 5][i & 31]),
-                                   __uint_as_float(r[i >> 5][(i & 31) + 1]));
-        const float mx =
-            fmax3(fmax3(mc[0], mc[1], mc[2]), fmax3(mc[3], mc[4], mc[5]), fmaxf(mc[6], mc[7]));
+        for (int i = 0; i < HB; ++i) mc[i % 16] = fmaxf(mc[i % 16], __uint_as_float(r[i >> 5][i & 31]));
+#pragma unroll
+        for (int w = 8; w >= 1; w >>= 1)
+#pragma unroll
+          for (int k = 0; k < w; ++k) mc[k] = fmaxf(mc[k], mc[k + w]);
+        const float mx = mc[0];
         const float m_new = fmaxf(m, mx * p.sl2);
         // Lazy rescale: keep a stale maximum unless the new one exceeds it
         // by more than 2^8 (probabilities then stay below 256).
@@ -516,7 +516,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // (a row that has seen no key yet keeps m = -inf: its P is 0)
         const float mneg = m == -INFINITY ? 0.f : -m;
         const float2 sl2v = make_float2(p.sl2, p.sl2), negm = make_float2(mneg, mneg);
-        float2 rs[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+        float2 rs[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
           uint32_t pk[16];
@@ -532,12 +532,12 @@ __global__ void __launch_bounds__(kThreads, 1)
               pv.x = ex2_mufu(a.x);
               pv.y = ex2_mufu(a.y);
             }
-            rs[pr_i & 1] = fadd2(rs[pr_i & 1], pv);
+            rs[pr_i & 3] = fadd2(rs[pr_i & 3], pv);
             pk[e >> 1] = f2_to_bf2(pv.x, pv.y);
           }
           tmem_st16(t_S + hf * HB + c * 16, pk);
         }
-        l += (rs[0].x + rs[0].y) + (rs[1].x + rs[1].y);
+        l += ((rs[0].x + rs[0].y) + (rs[1].x + rs[1].y)) + ((rs[2].x + rs[2].y) + (rs[3].x + rs[3].y));
         // O_h rescale for rows whose maximum moved (rare).  The previous tile's O += P V may still run: wait for it
         // (pv_done completes once per product, so its phase g - 1 is that
         // one); this tile's is not issued before p_full.

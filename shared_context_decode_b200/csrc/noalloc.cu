@@ -21,6 +21,8 @@
 // start at zero (each call writes every partial it later reads), but calls
 // whose kernels overlap on the GPU overwrite each other's partials: the caller
 // must order them (one stream, or events).
+#include <nvtx3/nvToolsExt.h>
+
 #include <atomic>
 #include <mutex>
 
@@ -53,10 +55,11 @@ pp_status scratch_address(void** out) {
 
 }  // namespace
 
-extern "C" __attribute__((visibility("default"))) pp_status pp_decode_attn_noalloc(
-    const pp_kv_layer* layer, int32_t doc_len, const uint16_t* q, const int16_t* q_sid,
-    const int32_t* q_pos, int32_t P, float scale, uint16_t* o, float* lse, const pp_options* opt,
-    void* stream) {
+namespace {
+
+pp_status decode_noalloc(const pp_kv_layer* layer, int32_t doc_len, const uint16_t* q,
+                         const int16_t* q_sid, const int32_t* q_pos, int32_t P, float scale,
+                         uint16_t* o, float* lse, const pp_options* opt, void* stream) {
   // The argument errors pp_decode_attn reports come first, with its codes.
   const pp_status v = pp::check_layer(layer);
   if (v != PP_OK) return v;
@@ -70,4 +73,16 @@ extern "C" __attribute__((visibility("default"))) pp_status pp_decode_attn_noall
   if (s != PP_OK) return s;
   return pp_decode_attn(layer, doc_len, q, q_sid, q_pos, P, scale, o, lse, scratch,
                         PP_NOALLOC_SCRATCH_BYTES, opt, stream);
+}
+
+}  // namespace
+
+extern "C" __attribute__((visibility("default"))) pp_status pp_decode_attn_noalloc(
+    const pp_kv_layer* layer, int32_t doc_len, const uint16_t* q, const int16_t* q_sid,
+    const int32_t* q_pos, int32_t P, float scale, uint16_t* o, float* lse, const pp_options* opt,
+    void* stream) {
+  nvtxRangePushA("pp_decode_attn_noalloc");
+  const pp_status st = decode_noalloc(layer, doc_len, q, q_sid, q_pos, P, scale, o, lse, opt, stream);
+  nvtxRangePop();
+  return st;
 }

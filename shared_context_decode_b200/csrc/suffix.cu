@@ -13,8 +13,11 @@
 // contiguous), NS-1 chunks ahead of the warp and across item boundaries.
 //
 // Balance: segments differ in length (questions and answers of different
-// lengths), so equal item counts per warp leave the slowest warp with far
-// more chunks than the mean.  With up to kBalanceRows rows each CTA first
+// lengths), so equal item counts per warp leave the slowest warp with more
+// chunks than the mean (29 against 21 at 256 streams, 32 heads).  Each
+// item's head and row go into the warp's item table once, so the per-chunk
+// path does no index division.  Slices balanced by work: with up to
+// kBalanceRows rows each CTA first
 // counts every item's work in units (its chunks, at least one for the merge)
 // and the warps take equal slices of the head-major unit sequence.  An item
 // cut by a slice boundary gets a partial (m, l, o) from each warp it spans;
@@ -54,11 +57,11 @@ struct SufCfg {
   static constexpr int STAGE = 2 * HALF;
   static constexpr int NS = 2;               // stages per warp (NS-1 chunks in flight)
   static constexpr int WARPS = kSuffixWarps;  // warps per CTA
-  static constexpr int TBL = BAL ? 32 : 128;  // item-table entries per warp and round
-  static constexpr int PRE = 4;              // document partials prefetched per lane
+  static constexpr int TBL = BAL ? 32 : 64;   // item-table entries per warp and round
+  static constexpr int PRE = 8;              // document partials prefetched per lane
   static constexpr int G = D / 64;           // 16-byte groups per lane and key row
   static constexpr int E = D / 32;           // output dims per lane
-  static constexpr int TBL_BYTES = WARPS * TBL * (BAL ? 24 : 16);   // ItemRec tables
+  static constexpr int TBL_BYTES = WARPS * TBL * (BAL ? 28 : 20);   // ItemRec tables
   static constexpr int PRE_BYTES = BAL ? (kBalanceRows + 1) * 4 : 0;  // units prefix over rows
   static constexpr int SMEM = WARPS * NS * STAGE + TBL_BYTES + PRE_BYTES + 128;
   static_assert(SMEM <= 227 * 1024, "dynamic shared memory above the per-CTA limit");
@@ -95,11 +98,11 @@ struct SufParams {
 
 // Per-item record of the warp's table: stream id (0 when the row is not an
 // answer-stream query), query position, visible-segment length, raw stream
-// id; balanced slices add the keys [tb, te) of the segment this warp covers
-// (else the whole segment).
+// id, head << 16 | row; balanced slices add the keys [tb, te) of the segment
+// this warp covers (else the whole segment).
 template <bool BAL>
 struct ItemRec {
-  int s, qp, n, raw;
+  int s, qp, n, raw, hr;
   __device__ int tb() const { return 0; }
   __device__ int te() const { return n; }
   __device__ void set_range(int, int) {}
@@ -107,13 +110,13 @@ struct ItemRec {
 };
 template <>
 struct ItemRec<true> {
-  int s, qp, n, raw, tb_, te_;
+  int s, qp, n, raw, hr, tb_, te_;
   __device__ int tb() const { return tb_; }
   __device__ int te() const { return te_; }
   __device__ void set_range(int b, int e) { tb_ = b; te_ = e; }
   __device__ void clamp_range() { te_ = te_ < n ? te_ : n; }
 };
-static_assert(sizeof(ItemRec<false>) == 16 && sizeof(ItemRec<true>) == 24, "table entry size");
+static_assert(sizeof(ItemRec<false>) == 20 && sizeof(ItemRec<true>) == 28, "table entry size");
 
 // Online-softmax state fold: (m, l, a) <- (m, l, a) (+) (m2, l2, a2).
 __device__ __forceinline__ void fold(float& m, float& l, float (&a)[8], float m2, float l2,
@@ -271,8 +274,10 @@ __global__ void __launch_bounds__(SufCfg<D, BAL>::WARPS * 32) suffix_merge(const
     if (u == S || U > kSnapUnits) return u;
     return (u - S) * 2 <= U ? S : S + U;
   };
-  // this warp's items, first .. last inclusive, and (balanced) its units
-  int64_t i_first, i_last, u_lo = 0, u_hi = 0;
+  // this warp's items, a contiguous range of the head-major items
+  // (h * rows + r): n_w of them, hr_at(k) giving the k-th as head << 16 |
+  // row; balanced: also its units
+  int64_t i_first = 0, i_last = -1, u_lo = 0, u_hi = 0, n_w = 0;
   if constexpr (balanced) {
     u_lo = gw < GWe ? snap(gw * T / GWe) : 0;
     u_hi = gw < GWe ? snap((gw + 1) * T / GWe) : 0;
@@ -282,27 +287,34 @@ __global__ void __launch_bounds__(SufCfg<D, BAL>::WARPS * 32) suffix_merge(const
     i_first = gw * items / GW;
     i_last = (gw + 1) * items / GW - 1;
   }
+  n_w = i_last - i_first + 1;
+  auto hr_at = [&](int64_t k) -> int {
+    const int64_t item = i_first + k;
+    const int h = (int)(item / p.rows);
+    return (h << 16) | (int)(item - (int64_t)h * p.rows);
+  };
 
   // each segment is read once, so its lines go first and the document
   // partials the merge reads stay in L2
   const uint64_t pol = l2_policy_evict_first();
   uint32_t issued = 0, consumed = 0;
   bool ok = true;
-  for (int64_t r0 = i_first; ok && r0 <= i_last; r0 += C::TBL) {
-    const int cnt = (int)min((int64_t)C::TBL, i_last - r0 + 1);
+  for (int64_t k0 = 0; ok && k0 < n_w; k0 += C::TBL) {
+    const int cnt = (int)min((int64_t)C::TBL, n_w - k0);
     // ---- item table of this round: two parallel gathers instead of one
     // dependent chain per item
     for (int k = lane; k < cnt; k += 32) {
-      const int64_t item = r0 + k;
-      const int r = (int)(item % p.rows);
+      const int hr = hr_at(k0 + k);
+      const int r = hr & 0xffff;
       const int s = p.q_sid[r];
       Rec rec;
+      rec.hr = hr;
       rec.qp = p.q_pos[r];
       rec.s = stream_query(s, p.P_max) ? s : 0;
       rec.n = 0;
       rec.raw = s;
       if constexpr (balanced) {  // this warp's units of the item, as keys
-        const int64_t S = (int64_t)((int)item / p.rows) * Ctot + pre[r];  // items < 2^31
+        const int64_t S = (int64_t)(hr >> 16) * Ctot + pre[r];
         const int64_t U = pre[r + 1] - pre[r];
         rec.set_range((int)((u_lo > S ? u_lo - S : 0) * C::CK),
                       (int)((u_hi < S + U ? u_hi - S : U) * C::CK));
@@ -315,9 +327,9 @@ __global__ void __launch_bounds__(SufCfg<D, BAL>::WARPS * 32) suffix_merge(const
       if (s) {
         int n;
         if (p.row_len) {
-          const int64_t item = r0 + k;
-          n = p.row_len[item % p.rows];
-          if (item < p.rows) p.len[s - 1] = n;   // head 0's items store the advanced length
+          const int hr = tbl[k].hr;
+          n = p.row_len[hr & 0xffff];
+          if ((hr >> 16) == 0) p.len[s - 1] = n;   // head 0's items store the advanced length
         } else {
           n = p.len[s - 1];
         }
@@ -337,7 +349,7 @@ __global__ void __launch_bounds__(SufCfg<D, BAL>::WARPS * 32) suffix_merge(const
       if (pk >= cnt) return false;
       if (lane == 0) {
         const Rec rec = tbl[pk];
-        const int h = (int)((r0 + pk) / p.rows);
+        const int h = rec.hr >> 16;
         const size_t seg = ((size_t)(rec.s - 1) * p.H + h) * seg_elems + (size_t)pt0 * D;
         const int nk = min(C::CK, rec.te() - pt0);
         uint8_t* st = ring + stage * C::STAGE;
@@ -357,8 +369,7 @@ __global__ void __launch_bounds__(SufCfg<D, BAL>::WARPS * 32) suffix_merge(const
     uint4 qn[C::G];
     int sid0 = -1, pos0 = 0;
     auto prefetch_item = [&](int k) {
-      const int64_t item = r0 + k;
-      const int h = (int)(item / p.rows), r = (int)(item - (int64_t)h * p.rows);
+      const int h = tbl[k].hr >> 16, r = tbl[k].hr & 0xffff;
       const uint4* qp4 = reinterpret_cast<const uint4*>(p.q + ((int64_t)r * p.H + h) * D);
 #pragma unroll
       for (int c = 0; c < C::G; ++c) qn[c] = __ldg(qp4 + g + 8 * c);
@@ -373,9 +384,9 @@ __global__ void __launch_bounds__(SufCfg<D, BAL>::WARPS * 32) suffix_merge(const
     if (cnt > 0) prefetch_item(0);
 
     for (int k = 0; k < cnt; ++k) {
-      const int64_t item = r0 + k;
-      const int h = (int)(item / p.rows), r = (int)(item - (int64_t)h * p.rows);
+      const int64_t item = i_first + k0 + k;   // balanced slices only
       const Rec rec = tbl[k];
+      const int h = rec.hr >> 16, r = rec.hr & 0xffff;
       uint4 qr[C::G];
 #pragma unroll
       for (int c = 0; c < C::G; ++c) qr[c] = qn[c];

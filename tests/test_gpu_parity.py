@@ -47,20 +47,20 @@ def test_ragged_two_mtiles_split_variants(splits):
 
 @pytest.mark.parametrize("P", [64, 128])
 @pytest.mark.parametrize("splits", [1, 3, 7, 20, 32])
-def test_single_mtile_tile_parity_split(P, splits):
-    """Row groups with one M tile: the two softmax warpgroups take alternate
-    key tiles of it and combine at the end of each segment, including
-    segments of one tile (the second warpgroup then has none) and of odd
-    length; 8 key tiles with a 104-key tail, 4 heads."""
+def test_single_mtile_many_splits(P, splits):
+    """Row groups of at most 128 rows (one M tile, one CTA per slot) under
+    split counts from one slot to one key tile per slot, so segments of one
+    tile and of odd length occur; 8 key tiles with a 104-key tail, 4 heads."""
     W = wl.make_decode(layers=1, H=4, d=128, N=1000, P=P, q=(1, 20), a=(0, 10), seed=31,
                        device=DEV)
     decode_case(W, opt=gu.pp().Options(splits=splits))
 
 
 @pytest.mark.parametrize("splits", [1, 4, 9, 25, 33])
-def test_mixed_mtile_modes_across_segments(splits):
+def test_mixed_row_group_sizes_across_segments(splits):
     """P = 300: the first row group has two M tiles, the second one (44 rows)
-    only one, so CTAs cross between the two modes of the document pass."""
+    only one, so a slot's CTA pair crosses from a full group into one whose
+    second M tile is empty."""
     W = wl.make_decode(layers=1, H=3, d=128, N=1000, P=300, q=(1, 9), a=(0, 4), seed=32,
                        device=DEV)
     decode_case(W, opt=gu.pp().Options(splits=splits))
@@ -110,11 +110,10 @@ def test_inactive_rows_are_zero():
 
 @pytest.mark.parametrize("P,H,d,a,active_every", [(300, 16, 128, (0, 40), 3), (5000, 1, 64, (0, 20), 0),
                                                   (257, 14, 128, (0, 63), 0)])
-def test_equal_item_counts_longest_first(P, H, d, a, active_every):
-    """The suffix pass with equal item counts per warp: each CTA sorts the
-    rows by work and deals the items longest first.  Inactive rows (no work,
-    sorted last), a row count above the sorted limit (contiguous items
-    instead) and a ragged head count."""
+def test_equal_item_counts_per_warp(P, H, d, a, active_every):
+    """The suffix pass with equal item counts per warp on inactive rows
+    mixed with active ones, more rows than the balanced mode takes, and a
+    head count that leaves a ragged last warp."""
     m = gu.pp()
     W = wl.make_decode(layers=1, H=H, d=d, N=300, P=P, q=(1, 20), a=a, seed=33, device=DEV)
     active = (np.arange(P) % active_every != 1) if active_every else None
@@ -126,7 +125,7 @@ def test_equal_item_counts_longest_first(P, H, d, a, active_every):
     torch.cuda.synchronize()
     assert m.device_status(layer) == 0
     o_ref, lse_ref, _ = gu.oracle_decode(W, L)
-    gu.compare(o, lse, o_ref, lse_ref, "longest first")
+    gu.compare(o, lse, o_ref, lse_ref, "equal item counts")
 
 
 def test_doc_pass_stays_in_segment_when_other_streams_longer():

@@ -10,12 +10,13 @@ stream keeps its row with stream id -1 (no append, no suffix work).  Every
 step has its own decode tokens, copied into the graph's input buffers before
 the replay, as a generation loop does.
 
-After every step the cache bookkeeping (segment lengths, stream ids,
-positions and the K/V bits of every slot) must equal the append replay bit
-for bit, and stopped rows must give exactly zero.  On a seeded set of steps
-(the first, the first with a stopped stream, a middle one and the last) o
-and lse of every row and head must match the oracle over the replayed cache
-within the stated bar.
+After every step the segment lengths and the slot each active stream just
+gained (its stream id, position and K/V bits) must equal the append replay
+bit for bit, and stopped rows must give exactly zero.  On a seeded set of
+steps (the first, the first with a stopped stream, a middle one and the
+last) the whole cache (every slot's tags and K/V bits) must equal the
+replay, and o and lse of every row and head must match the oracle over the
+replayed cache within the stated bar.
 """
 import math
 
@@ -59,6 +60,29 @@ def check_state(layer, rep, what):
     assert np.array_equal(layer.pos.cpu().numpy(), pos), f"{what}: slot positions"
     assert np.array_equal(bf16_bits(layer.k_suf), k), f"{what}: slot keys"
     assert np.array_equal(bf16_bits(layer.v_suf), v), f"{what}: slot values"
+
+
+def check_new_slots(layer, rep, before, active, what):
+    """Lengths of every stream, and the slot each active stream gained in
+    this step, against the replay (its last slot)."""
+    ln = layer.len.cpu().numpy()
+    want = np.array([rep.length(s) for s in range(1, rep.P_max + 1)], np.int32)
+    assert np.array_equal(ln, want), f"{what}: segment lengths"
+    idx_s = np.nonzero(active)[0]
+    if idx_s.size == 0:
+        return
+    idx_t = before[idx_s]
+    dev = layer.len.device
+    si, ti = torch.from_numpy(idx_s).to(dev), torch.from_numpy(idx_t.astype(np.int64)).to(dev)
+    sid = layer.sid[si, ti].cpu().numpy()
+    pos = layer.pos[si, ti].cpu().numpy()
+    k = bf16_bits(layer.k_suf[si, :, ti, :])
+    v = bf16_bits(layer.v_suf[si, :, ti, :])
+    for n, s in enumerate(idx_s + 1):
+        kk, vv, ss, pp = rep.seg[s][-1]
+        assert sid[n] == ss and pos[n] == pp, f"{what}: tags of stream {s}'s new slot"
+        assert np.array_equal(k[n], kk) and np.array_equal(v[n], vv), \
+            f"{what}: K/V bits of stream {s}'s new slot"
 
 
 def oracle_step(rep, doc_k, doc_v, N, q, q_sid, q_pos, scale):
@@ -165,13 +189,16 @@ def test_sweep_graph_steps_match_oracle(N, P, layers, fused):
             for n in ("k", "v", "q"):
                 x[n].copy_(wl.randn_bf16((P, H, d), wl.seed_of(name, l, t, n), DEV))
             host.append({n: bf16_bits(x[n]) for n in ("k", "v", "q")})
+        before = [c.len.cpu().numpy().copy() for c in caches]
         g.replay()
         torch.cuda.synchronize()
         for l in range(layers):
             kv, rep, hx = caches[l], reps[l], host[l]
             rep.append(hx["k"], hx["v"], sid_t, pos_t)
             assert m.device_status(kv) == 0, f"step {t} layer {l}: device status"
-            check_state(kv, rep, f"step {t} layer {l}")
+            check_new_slots(kv, rep, before[l], active, f"step {t} layer {l}")
+            if t in checked:
+                check_state(kv, rep, f"step {t} layer {l}")
             o = bufs[l]["o"]
             assert torch.count_nonzero(o[torch.from_numpy(~active).to(DEV)]) == 0, \
                 f"step {t} layer {l}: stopped rows must give zero output"
