@@ -140,6 +140,18 @@ __device__ __forceinline__ bool next_seg(const DocTcParams& p, int64_t& t, int64
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                           long long limit, int32_t* status) {
   const int lane = threadIdx.x & 31;
+  {
+    // fast path: a phase that has already completed costs one non-blocking
+    // test, no clock read and no suspension
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    if (__all_sync(0xffffffffu, done != 0)) return true;
+  }
   const long long t0 = clock64();
   while (true) {
     const bool ok = mbar_try_wait_sleep(bar, parity, 20000);

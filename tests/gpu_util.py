@@ -7,8 +7,8 @@ import oracle
 from shared_context_decode_b200.workloads import bf16_bits
 from tests.flat import decode_slots, decode_queries, prefill_slots, prefill_queries
 
-# Tolerances on o (bf16 inputs, fp32 accumulation), from the north-star
-# statement of the method's acceptance bar: max |err| <= 1e-2, mean <= 1e-3.
+# Tolerances on o (bf16 inputs, fp32 accumulation), the method's acceptance
+# bar for this path: max |err| <= 1e-2, mean <= 1e-3.
 O_MAX, O_MEAN = 1e-2, 1e-3
 # lse is fp32 from fp32 scores of exact bf16 products.
 LSE_MAX = 5e-3
