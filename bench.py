@@ -555,6 +555,26 @@ def mode_docprefill(args, world, rank, local, dev):
     del step.graph
 
 
+def sweep_roof_ms(W, stops, steps: int, layers: int, peaks) -> float:
+    """Roof time of one sweep combination: per step, the slower of its
+    algorithmic bytes at the HBM copy rate and its FLOPs at the burst bf16
+    rate, summed over the steps.  Bytes per layer: the document K/V once,
+    every active stream's segment once (question, answers so far, the new
+    token), the new tokens' K/V read and written, q read and o written;
+    FLOPs: S = QK^T and O = PV of the active rows over the document and
+    their segments.  A stream is active at step t iff t < its stop length."""
+    N, P = W.N, W.P
+    kvb = W.H * W.d * 2 * 2
+    roof_ms = 0.0
+    for t in range(steps):
+        act = t < stops
+        seg_tok = float(((W.q_len + t + 1) * act).sum())
+        byt = layers * (N * kvb + seg_tok * kvb + 2 * int(act.sum()) * kvb + P * kvb)
+        fl = layers * 4.0 * W.d * W.H * (int(act.sum()) * N + seg_tok)
+        roof_ms += max(byt / (peaks["hbm"] * 1e9), fl / (peaks["bf16"] * 1e12)) * 1e3
+    return roof_ms
+
+
 def sweep_combo(N: int, P: int, layers: int, dev, warm: bool = True):
     """One doc x streams combination of the answer-generation sweep: returns
     (active stream-tokens, device ms) over its decode steps.  The graph holds
@@ -590,21 +610,7 @@ def sweep_combo(N: int, P: int, layers: int, dev, warm: bool = True):
     host = [(torch.from_numpy(np.where(t < stops, sids, -1).astype(np.int16)).pin_memory(),
              torch.from_numpy(base_pos + t).pin_memory(), int((t < stops).sum()))
             for t in range(steps)]
-    # Roof time of the combo: per step, the slower of its algorithmic bytes
-    # at the HBM copy rate and its FLOPs at the burst bf16 rate.  Bytes per
-    # layer: the document K/V once, every active stream's segment once
-    # (question, answers so far, the new token), the new tokens' K/V read and
-    # written, q read and o written; FLOPs: S = QK^T and O = PV of the
-    # active rows over the document and their segments.
-    peaks = load_peaks()
-    kvb = W.H * W.d * 2 * 2
-    roof_ms = 0.0
-    for t in range(steps):
-        act = t < stops
-        seg_tok = float(((W.q_len + t + 1) * act).sum())
-        byt = layers * (N * kvb + seg_tok * kvb + 2 * int(act.sum()) * kvb + P * kvb)
-        fl = layers * 4.0 * W.d * W.H * (int(act.sum()) * N + seg_tok)
-        roof_ms += max(byt / (peaks["hbm"] * 1e9), fl / (peaks["bf16"] * 1e12)) * 1e3
+    roof_ms = sweep_roof_ms(W, stops, steps, layers, load_peaks())
 
     def body():
         for l in range(layers):

@@ -5,6 +5,7 @@ import os
 import socket
 import sys
 
+import numpy as np
 import pytest
 import torch
 import torch.multiprocessing as mp
@@ -127,3 +128,25 @@ def test_doc_roofline_uses_the_burst_peak_and_reports_the_stricter_gate():
     r2 = bench.doc_roofline(W2, {"doc": 0.030, "suffix": 0.010}, peaks, None)
     assert r2["bound"] == "hbm" and r2["unit"] == "GB/s"
     assert r2["frac"] == pytest.approx((2 * 8192 * 32 * 128 * 2 / 6548e9) / 30e-6)
+
+
+def test_sweep_roof_time_by_hand():
+    """The sweep's roof time on a two-stream, two-step case worked by hand:
+    step 0 both streams active, step 1 only stream 1."""
+    sys.path.insert(0, ROOT)
+    import bench
+
+    class W:
+        N, P, H, d = 1000, 2, 4, 64
+        q_len = np.array([10, 20])
+
+    peaks = dict(hbm=1000.0, bf16=1000.0)
+    kvb = 4 * 64 * 2 * 2
+    # step 0: segments 11 + 21 tokens; step 1: stream 1 only, 12 tokens
+    b0 = 3 * (1000 * kvb + 32 * kvb + 2 * 2 * kvb + 2 * kvb)
+    f0 = 3 * 4.0 * 64 * 4 * (2 * 1000 + 32)
+    b1 = 3 * (1000 * kvb + 12 * kvb + 2 * 1 * kvb + 2 * kvb)
+    f1 = 3 * 4.0 * 64 * 4 * (1 * 1000 + 12)
+    want = sum(max(b / 1e12, f / 1e15) for b, f in ((b0, f0), (b1, f1))) * 1e3
+    got = bench.sweep_roof_ms(W, np.array([2, 1]), 2, 3, peaks)
+    assert got == pytest.approx(want)
