@@ -659,6 +659,7 @@ def sweep_combo(N: int, P: int, layers: int, dev, warm: bool = True):
 def mode_sweep(args, world, rank, local, dev):
     from shared_context_decode_b200 import workloads as wl
     nl = args.layers or 32
+    peaks = load_peaks()
     rows, tot_tok, tot_ms, tot_roof = [], 0, 0.0, 0.0
     with ClockSampler(local) as clocks:
         clocks.mark("start")
@@ -681,7 +682,7 @@ def mode_sweep(args, world, rank, local, dev):
                        "streams": list(wl.SWEEP_STREAMS),
                        "stops": f"min({wl.SWEEP_STOP_CAP}, Geometric(1/{wl.SWEEP_STOP_MEAN}))"},
             "roofline": {"roof_ms": tot_roof, "ms": tot_ms, "frac": tot_roof / tot_ms,
-                         "peaks": "measured HBM copy, burst bf16"},
+                         "peaks": f"HBM copy and burst bf16, {peaks['source']}"},
             "combos": rows, "clocks": clocks.summary()}
     if rank == 0:
         print(json.dumps(line), flush=True)
