@@ -116,14 +116,16 @@ SplitPlan plan_for(int rows, int H, int doc_len, const pp_options* opt, bool cau
 }
 
 struct WsLayout {
-  size_t doc_o, doc_ml, row_len, split_cnt, split_o, split_ml, total;
+  size_t doc_o, doc_ml, row_len, split_cnt, split_o, split_ml, runs, n_runs, total;
 };
 
 // The document pass leaves its partial results in the workspace.  Besides,
 // for decode and question prefill (not the causal document prefill): each
 // row's stream length when the pass carries a decode step's append, and the
-// decode suffix pass's counters and partials for items cut between warps.
-WsLayout ws_layout(const SplitPlan& p, int d) {
+// decode suffix pass's counters and partials for items cut between warps;
+// question prefill (questions = true): the question runs (at most one per
+// row) and their count.
+WsLayout ws_layout(const SplitPlan& p, int d, bool questions) {
   WsLayout w;
   const size_t slots = (size_t)p.units * p.max_chunks * pp::kGroupRows;
   const bool extra = slots && !p.causal;
@@ -134,7 +136,9 @@ WsLayout ws_layout(const SplitPlan& p, int d) {
   w.split_cnt = w.row_len + (extra ? up((size_t)p.G * pp::kGroupRows * sizeof(int32_t)) : 0);
   w.split_o = w.split_cnt + up(warps * sizeof(int32_t));
   w.split_ml = w.split_o + up(2 * warps * d * sizeof(float));
-  w.total = w.split_ml + up(2 * warps * 2 * sizeof(float));
+  w.runs = w.split_ml + up(2 * warps * 2 * sizeof(float));
+  w.n_runs = w.runs + (questions ? up((size_t)p.G * pp::kGroupRows * sizeof(int4)) : 0);
+  w.total = w.n_runs + (questions ? up(sizeof(int32_t)) : 0);
   return w;
 }
 
@@ -185,7 +189,7 @@ pp_status attend(const pp_kv_layer* L, int32_t doc_len, const uint16_t* q, const
   const SplitPlan plan = plan_for(rows, L->H, doc_len, opt, causal);
   const bool has_doc = doc_len > 0;
   if (has_doc && plan.C < 1) return PP_ERR_CUDA;  // no device to size the split for
-  const WsLayout w = ws_layout(plan, L->d);
+  const WsLayout w = ws_layout(plan, L->d, !causal && !read_once);
   if (w.total > 0 && (!ws || !aligned(ws, kAlign))) return PP_ERR_INVALID_ARG;
   if (ws_bytes < w.total) return PP_ERR_CAPACITY;
   const int sms = sm_count();
@@ -252,6 +256,14 @@ pp_status attend(const pp_kv_layer* L, int32_t doc_len, const uint16_t* q, const
                                                app.n ? app.row_len : nullptr,
                                                balance ? &split : nullptr, st))) != PP_OK)
       return s;
+  } else if (!causal) {
+    int4* runs = reinterpret_cast<int4*>(wsb + w.runs);
+    int32_t* n_runs = reinterpret_cast<int32_t*>(wsb + w.n_runs);
+    if ((s = from_cuda(pp::launch_question_runs(*L, q_sid, rows, runs, n_runs, st))) != PP_OK)
+      return s;
+    if ((s = from_cuda(pp::launch_question_attn(*L, q, q_sid, q_pos, rows, scale, plan, has_doc,
+                                                part, o, lse, runs, n_runs, sms, st))) != PP_OK)
+      return s;
   } else if ((s = from_cuda(pp::launch_suffix_block(*L, q, q_sid, q_pos, rows, scale, plan,
                                                     has_doc, part, o, lse, sms, st))) != PP_OK) {
     return s;
@@ -259,12 +271,14 @@ pp_status attend(const pp_kv_layer* L, int32_t doc_len, const uint16_t* q, const
   return from_cuda(mark(2));
 }
 
+// questions: a question prefill (pp_prefill_attn), whose question runs
+// need room whether or not there is a document.
 size_t workspace(int32_t rows, int32_t H, int32_t d, int32_t doc_len, const pp_options* opt,
-                 bool causal = false) {
+                 bool causal = false, bool questions = false) {
   if (rows < 0 || H < 1 || (d != 64 && d != 128) || doc_len < 0) return 0;
   const SplitPlan plan = plan_for(rows, H, doc_len, opt, causal);
   if (doc_len > 0 && plan.C < 1) return 0;
-  return ws_layout(plan, d).total;
+  return ws_layout(plan, d, questions).total;
 }
 
 // Host copy of a plan for the split-plan test aids.
@@ -343,7 +357,7 @@ PP_API size_t pp_decode_workspace_bytes(int32_t P, int32_t H, int32_t d, int32_t
 
 PP_API size_t pp_prefill_workspace_bytes(int32_t R, int32_t H, int32_t d, int32_t doc_len,
                                   const pp_options* opt) {
-  return workspace(R, H, d, doc_len, opt);
+  return workspace(R, H, d, doc_len, opt, false, true);
 }
 
 PP_API pp_status pp_decode_attn(const pp_kv_layer* layer, int32_t doc_len, const uint16_t* q,

@@ -67,6 +67,16 @@ cudaError_t launch_suffix_block(const pp_kv_layer& L, const uint16_t* q, const i
                                 const int32_t* q_pos, int rows, float scale, const SplitPlan& plan,
                                 bool has_doc, const Partials& part, uint16_t* o, float* lse,
                                 int num_sms, cudaStream_t st);
+// Question part of a prefill call: the runs of consecutive rows with one
+// stream id (one block; runs[k] = first row, end row, stream id, visible
+// segment keys), then one warp per (run, head) with the merge first.
+cudaError_t launch_question_runs(const pp_kv_layer& L, const int16_t* q_sid, int rows, int4* runs,
+                                 int32_t* n_runs, cudaStream_t st);
+cudaError_t launch_question_attn(const pp_kv_layer& L, const uint16_t* q, const int16_t* q_sid,
+                                 const int32_t* q_pos, int rows, float scale, const SplitPlan& plan,
+                                 bool has_doc, const Partials& part, uint16_t* o, float* lse,
+                                 const int4* runs, const int32_t* n_runs, int num_sms,
+                                 cudaStream_t st);
 cudaError_t launch_visibility(const pp_kv_layer& L, int doc_len, const int16_t* q_sid,
                               const int32_t* q_pos, int nq, int32_t* count_out, uint8_t* mask_out,
                               cudaStream_t st);

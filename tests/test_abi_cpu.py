@@ -146,6 +146,11 @@ def test_workspace_sizes_with_explicit_split(pp):
     # (rounded up to whole row groups) for a step whose append the pass carries
     expect = slots * 128 * 4 + slots * 2 * 4 + groups * 256 * 4
     assert ws == expect
+    # a question prefill adds its question runs: 16 bytes a row (whole row
+    # groups) and their count in one 256-byte-aligned word, with a document
+    # or without one
+    assert pp.prefill_workspace_bytes(256, 32, 128, 16384, opt) == expect + groups * 256 * 16 + 256
+    assert pp.prefill_workspace_bytes(300, 2, 64, 0, opt) == 2 * 256 * 16 + 256
     assert pp.decode_workspace_bytes(4, 4, 96, 10, opt) == 0
     # no document: nothing to carry between kernels
     assert pp.decode_workspace_bytes(8, 2, 64, 0, opt) == 0
