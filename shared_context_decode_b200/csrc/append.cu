@@ -71,20 +71,21 @@ __global__ void __launch_bounds__(128) kv_append_rows(pp_kv_layer L, const uint4
   }
 }
 
-// Every accepted stream row advances its segment length by one, saturating
-// at S_cap (a compare-and-swap loop, so overflowed rows do not count).
+// Every stream row advances its segment length by one, saturating at S_cap:
+// an add, then a min with S_cap, from each row.  Whatever the order of the
+// rows' atomics, the last one on a length is a min, and the length ends at
+// min(S_cap, old + rows of the stream) -- exactly the rows kv_append_rows
+// accepted (rank < S_cap - old).  Neither atomic returns a value, so no row
+// waits on another (a compare-and-swap loop serialised the ~30 rows of a
+// question into round trips).
 __global__ void __launch_bounds__(256) kv_append_len(pp_kv_layer L, const int16_t* __restrict__ sid,
                                                      int n) {
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
     const int s = sid[i];
     if (s < 1 || s > L.P_max) continue;
     int* len = L.len + (s - 1);
-    int old = *reinterpret_cast<volatile int*>(len);
-    while (old < L.S_cap) {
-      const int seen = atomicCAS(len, old, old + 1);
-      if (seen == old) break;
-      old = seen;
-    }
+    atomicAdd(len, 1);
+    atomicMin(len, L.S_cap);
   }
 }
 
