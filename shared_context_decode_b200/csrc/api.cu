@@ -264,9 +264,9 @@ pp_status attend(const pp_kv_layer* L, int32_t doc_len, const uint16_t* q, const
     if ((s = from_cuda(pp::launch_question_attn(*L, q, q_sid, q_pos, rows, scale, plan, has_doc,
                                                 part, o, lse, runs, n_runs, sms, st))) != PP_OK)
       return s;
-  } else if ((s = from_cuda(pp::launch_suffix_block(*L, q, q_sid, q_pos, rows, scale, plan,
-                                                    has_doc, part, o, lse, sms, st))) != PP_OK) {
-    return s;
+  } else if ((s = from_cuda(pp::launch_doc_merge(rows, L->H, L->d, plan, part, o, lse, st))) !=
+             PP_OK) {
+    return s;  // a document prefill: its rows see the document only
   }
   return from_cuda(mark(2));
 }

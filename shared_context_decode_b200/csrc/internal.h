@@ -61,12 +61,10 @@ cudaError_t launch_suffix_merge(const pp_kv_layer& L, const uint16_t* q, const i
                                 bool has_doc, const Partials& part, uint16_t* o, float* lse,
                                 long long wait_limit, int num_sms, const int32_t* row_len,
                                 const SuffixSplit* split, cudaStream_t st);
-// Suffix pass of a prefill call (one warp per 16 rows and head, warp-level
-// mma), merge first; q_sid = nullptr for document rows.  Writes o and lse.
-cudaError_t launch_suffix_block(const pp_kv_layer& L, const uint16_t* q, const int16_t* q_sid,
-                                const int32_t* q_pos, int rows, float scale, const SplitPlan& plan,
-                                bool has_doc, const Partials& part, uint16_t* o, float* lse,
-                                int num_sms, cudaStream_t st);
+// Merge of a document prefill (rows = document tokens): each row's document
+// partials combined into o and lse, one warp per row and head.
+cudaError_t launch_doc_merge(int rows, int H, int d, const SplitPlan& plan, const Partials& part,
+                             uint16_t* o, float* lse, cudaStream_t st);
 // Question part of a prefill call: the runs of consecutive rows with one
 // stream id (one block; runs[k] = first row, end row, stream id, visible
 // segment keys), then one warp per (run, head) with the merge first.

@@ -5,7 +5,7 @@
 // project page, section "How it works", item 1: same stream id and not later
 // than the query).  This kernel serves decode steps (one row per stream, so
 // every segment is read by one row); prefill calls, whose rows share their
-// question's segment, run the question-block kernel of suffix_block.cu.
+// question's segment, run the question kernel of question.cu.
 //
 // Work item = (query row, head).  Each warp owns a contiguous slice of the
 // items and a ring of NS shared-memory stages; lane 0 fills them with 1-D
