@@ -1,8 +1,10 @@
 """Prefill calls against the oracle on layouts the named workloads do not
-reach: streams interleaved inside a block of 16 rows, segments longer than
-one 32-key chunk, follow-up questions behind cached answers (rows whose
-segment holds earlier tokens), inactive and out-of-range rows, d = 64, no
-document, row counts that leave a ragged last block.
+reach: rows of many streams interleaved (runs of one or two rows, a stream
+split into several runs), runs of many 16-row tiles over segments longer
+than one 48-key chunk, follow-up questions behind cached answers (rows whose
+segment holds earlier tokens), inactive and out-of-range rows inside runs,
+d = 64, no document, runs that cross a 256-row group of document partials,
+row counts that leave a ragged last tile.
 
 Visibility rule: project page "Read Once, Answer Many", section "How it
 works", item 1 -- a row sees the document and the tokens of its own stream
