@@ -120,8 +120,9 @@ typedef struct pp_kv_layer {
  *                           result, kept to measure what per-stream segments
  *                           save.  Decode and question prefill only.
  *   suffix_slices           decode suffix pass, how its warps share the (row,
- *                           head) items: 0 = automatic (balanced when there
- *                           are few items or segments may pass 512 keys),
+ *                           head) items: 0 = automatic (balanced when the
+ *                           items would keep fewer than half of the warps
+ *                           busy or segments may pass 512 keys),
  *                           1 = equal item counts, 2 = balanced by work (an
  *                           item longer than 8 chunks may be cut between
  *                           warps; needs the tensor-core document pass and

@@ -212,11 +212,13 @@ pp_status attend(const pp_kv_layer* L, int32_t doc_len, const uint16_t* q, const
   // balanced by work, with counters that pass zeroes
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   pp::SuffixSplit split{};
-  // automatic: when equal item counts would leave warps idle (fewer items
-  // than twice the warps) or a few long segments could hold most of the work
+  // automatic: when equal item counts would leave most warps idle (items
+  // for fewer than half of them) or a few long segments could hold most of
+  // the work.  (With about one item per warp equal counts measured faster:
+  // 22.5 against 26.7 us at 64 streams x 32 heads over 8192 document keys.)
   const int slices = opt ? opt->suffix_slices : 0;
   const bool want = slices == 2 ||
-                    (slices == 0 && ((int64_t)rows * L->H < 2LL * sms * pp::kSuffixWarps ||
+                    (slices == 0 && (2LL * rows * L->H < (int64_t)sms * pp::kSuffixWarps ||
                                      L->S_cap > 32 * 16));
   const bool balance = want && read_once && has_doc && !other_doc && rows <= pp::kBalanceRows &&
                        (int64_t)rows * L->H < (1LL << 31);
