@@ -267,7 +267,12 @@ pp_status pp_decode_attn_noalloc(const pp_kv_layer *layer, int32_t doc_len, cons
                                  float scale, uint16_t *o, float *lse, const pp_options *opt,
                                  void *stream);
 
-/* Workspace bytes pp_prefill_attn needs for R question rows. */
+/*
+ * Workspace bytes pp_prefill_attn needs for R question rows: the document
+ * pass's fp32 partial results (as for decode) and the question runs -- 16
+ * bytes a row (whole groups of 256 rows) and their count -- which are
+ * needed with or without a document.
+ */
 size_t pp_prefill_workspace_bytes(int32_t R, int32_t H, int32_t d, int32_t doc_len,
                                   const pp_options *opt);
 
@@ -276,7 +281,9 @@ size_t pp_prefill_workspace_bytes(int32_t R, int32_t H, int32_t d, int32_t doc_l
  * figure: the document and all questions go into one sequence, prefilled
  * once; each question gets its own answer stream that sees only the
  * document and its own question).
- *   q       bf16 [R][H][d]  question rows, any order
+ *   q       bf16 [R][H][d]  question rows, any order (a question's rows
+ *                           next to each other are read together: its
+ *                           segment is copied once for all of them)
  *   q_sid   int16 [R]       stream of each row (1..P_max; -1 = inactive)
  *   q_pos   int32 [R]       position of each row (N + index in its question)
  *   o bf16 [R][H][d], lse fp32 [R][H] or NULL, ws as for decode.
