@@ -204,7 +204,10 @@ __global__ void __launch_bounds__(QCfg<D>::WARPS * 32, 1) question_attn(const QP
         if (kk < C::KC) {
           const int t = t0 + kk;
           int kp = INT32_MAX;
-          if (t < n && tsid[t] == s) kp = tpos[t];
+          if (t < n) {  // both tags at once: one round trip, not two
+            const int sd = tsid[t], ps = tpos[t];
+            kp = sd == s ? ps : INT32_MAX;
+          }
           kpos[kk] = kp;
         }
       }
