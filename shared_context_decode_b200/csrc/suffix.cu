@@ -311,7 +311,11 @@ __global__ void __launch_bounds__(SufCfg<D, BAL>::WARPS * 32) suffix_merge(const
       rec.hr = hr;
       rec.qp = p.q_pos[r];
       rec.s = stream_query(s, p.P_max) ? s : 0;
-      rec.n = 0;
+      // a row's length left by the document pass's append needs no stream
+      // id: load it beside the tags (one round trip less); a row that is not
+      // an answer-stream query has no segment (0)
+      const int rl = p.row_len ? p.row_len[r] : 0;
+      rec.n = rec.s ? rl : 0;
       rec.raw = s;
       if constexpr (balanced) {  // this warp's units of the item, as keys
         const int64_t S = (int64_t)(hr >> 16) * Ctot + pre[r];
@@ -327,9 +331,8 @@ __global__ void __launch_bounds__(SufCfg<D, BAL>::WARPS * 32) suffix_merge(const
       if (s) {
         int n;
         if (p.row_len) {
-          const int hr = tbl[k].hr;
-          n = p.row_len[hr & 0xffff];
-          if ((hr >> 16) == 0) p.len[s - 1] = n;   // head 0's items store the advanced length
+          n = tbl[k].n;
+          if ((tbl[k].hr >> 16) == 0) p.len[s - 1] = n;   // head 0's items store the advanced length
         } else {
           n = p.len[s - 1];
         }
