@@ -703,32 +703,41 @@ def doc_pass_algorithmic(W):
 SPEC_HBM_GBS, SPEC_BF16_TFLOPS = 8000.0, 2250.0
 
 
-def doc_roofline(W, durs, peaks, traffic):
-    """Roofline record of the document pass.  Its time is measured over a
-    few replays of one step (milliseconds, not a seconds-long loop), so the
-    burst bf16 peak applies; the roof time is the slower of the algorithmic
-    bytes at the measured HBM copy rate and the FLOPs at that peak, and frac
-    is roof time / measured time.  The same fraction against the sustained
-    bf16 peak and against the nominal figures (8 TB/s, 2.25 PFLOP/s: the
-    stricter gate) is reported beside it."""
+def doc_roofline(W, durs, peaks, traffic, sustained: bool = False):
+    """Roofline record of the document pass.  The roof time is the slower of
+    the algorithmic bytes at the measured HBM copy rate and the FLOPs at the
+    bf16 tensor peak, and frac is roof time / measured time.  The tensor
+    peak is the burst one when the run was short and cool (timed region
+    under a second, no power cap in the clock samples), else the sustained
+    one (the rate a seconds-long loop under the power cap settles at):
+    sustained=True.  The fractions against both peaks and against the
+    nominal figures (8 TB/s, 2.25 PFLOP/s: the stricter gate) are reported
+    beside it."""
     b, f = doc_pass_algorithmic(W)
     t_doc = durs["doc"] * 1e-3
     gbs, tfs = b / t_doc / 1e9, f / t_doc / 1e12
-    t_hbm, t_tc = b / (peaks["hbm"] * 1e9), f / (peaks["bf16"] * 1e12)
+    bf16 = peaks["bf16_sustained"] if sustained else peaks["bf16"]
+    t_hbm, t_tc = b / (peaks["hbm"] * 1e9), f / (bf16 * 1e12)
     if t_tc > t_hbm:
-        roof = {"bound": "tensor", "achieved": tfs, "peak": peaks["bf16"], "unit": "TFLOP/s"}
+        roof = {"bound": "tensor", "achieved": tfs, "peak": bf16, "unit": "TFLOP/s"}
     else:
         roof = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm"], "unit": "GB/s"}
     roof["frac"] = max(t_hbm, t_tc) / t_doc
+    t_burst = f / (peaks["bf16"] * 1e12)
     t_sus = f / (peaks["bf16_sustained"] * 1e12)
     t_spec = max(b / (SPEC_HBM_GBS * 1e9), f / (SPEC_BF16_TFLOPS * 1e12))
+    tensor_peak = "sustained bf16" if sustained else "burst bf16"
     roof.update({"traffic": traffic, "kernel": f"pp::doc_pass_tc<{W.d}>",
-                 "peak_source": peaks["source"] + (" burst bf16" if roof["bound"] == "tensor"
+                 "peak_source": peaks["source"] + (" " + tensor_peak if roof["bound"] == "tensor"
                                                    else " copy"),
+                 "tensor_peak": tensor_peak,
+                 "peak_rule": "burst bf16 when the timed region is under 1 s and the clock "
+                              "samples show no power cap, else sustained bf16",
                  "roof_us": max(t_hbm, t_tc) * 1e6,
                  "doc_us": durs["doc"] * 1e3, "suffix_merge_us": durs["suffix"] * 1e3,
                  "doc_hbm_gbs": gbs, "doc_tflops": tfs,
                  "frac_hbm": gbs / peaks["hbm"], "frac_tensor_burst": tfs / peaks["bf16"],
+                 "frac_burst": max(t_hbm, t_burst) / t_doc,
                  "frac_sustained": max(t_hbm, t_sus) / t_doc,
                  "frac_spec": t_spec / t_doc,
                  "frac_gate": min(max(t_hbm, t_tc), t_spec) / t_doc})
@@ -1005,7 +1014,13 @@ def main():
 
     # ---- roofline of the dominant kernel (document pass), live CUDA events
     durs = measure_doc_pass(step, args.roofline_reps)
-    roof = doc_roofline(W, durs, load_peaks(), profile_traffic(doc_profile(args.workload)))
+    # the tensor peak the document pass is held to: burst for a short, cool
+    # run, sustained when the timed region lasted a second or more or the
+    # clocks were held down by the power cap
+    clk = clocks.summary()
+    sustained = args.steps * ms_rank >= 1000.0 or "sw_power_cap" in clk.get("reasons", [])
+    roof = doc_roofline(W, durs, load_peaks(), profile_traffic(doc_profile(args.workload)),
+                        sustained=sustained)
 
     cpu = None
     if rank == 0 and world == 1 and args.cpu_seconds > 0:

@@ -105,10 +105,11 @@ def test_profile_traffic_only_while_the_sources_match(tmp_path):
     assert bench.profile_traffic(str(tmp_path / "absent.md")) is None
 
 
-def test_doc_roofline_uses_the_burst_peak_and_reports_the_stricter_gate():
+def test_doc_roofline_peak_choice_and_the_stricter_gate():
     """The document pass's roofline: roof time = the slower of the bytes at
-    the measured copy rate and the FLOPs at the burst bf16 rate; frac = roof
-    time / measured time.  The nominal figures give the stricter gate."""
+    the measured copy rate and the FLOPs at the bf16 rate (burst for a short,
+    cool run; sustained for a long or power-capped one); frac = roof time /
+    measured time.  The nominal figures give the stricter gate."""
     sys.path.insert(0, ROOT)
     import bench
     from shared_context_decode_b200 import workloads as wl
@@ -123,6 +124,13 @@ def test_doc_roofline_uses_the_burst_peak_and_reports_the_stricter_gate():
     assert r["frac_spec"] == pytest.approx(max(b / 8e12, f / 2.25e15) / 72.5e-6)
     assert r["frac_gate"] == pytest.approx(min(r["frac"], r["frac_spec"]))
     assert r["frac_sustained"] > r["frac"]
+    assert r["frac_burst"] == pytest.approx(r["frac"]) and r["tensor_peak"] == "burst bf16"
+    # a long or power-capped run is held to the sustained peak
+    rs = bench.doc_roofline(W, {"doc": 0.0725, "suffix": 0.0594}, peaks, None, sustained=True)
+    assert rs["peak"] == 1390.0 and rs["tensor_peak"] == "sustained bf16"
+    assert rs["frac"] == pytest.approx(max(b / 6548e9, f / 1390e12) / 72.5e-6)
+    assert rs["frac"] == pytest.approx(r["frac_sustained"])
+    assert rs["frac_burst"] == pytest.approx(r["frac"])
     # a memory-bound workload (64 streams) is bound by HBM
     W2 = wl.make_decode("doc8k_p64", device="cpu")
     r2 = bench.doc_roofline(W2, {"doc": 0.030, "suffix": 0.010}, peaks, None)
