@@ -409,7 +409,7 @@ def mode_prefill(args, world, rank, local, dev):
     flops = 4.0 * W.R * W.N * W.d * W.H * nl
     tfs = flops / (ms / 1e3) / 1e12 * world
     peaks = load_peaks()
-    durs = measure_doc_pass(step, 2)          # per-layer document / suffix+merge times
+    durs = measure_doc_pass(step, 2)          # per-layer document pass / question part times
     doc_tfs = 4.0 * W.R * W.N * W.d * W.H / (durs["doc"] * 1e-3) / 1e12
     # question part + merge: segments read once, q read, o written, the
     # document partials (one chunk per row) read
@@ -423,7 +423,7 @@ def mode_prefill(args, world, rank, local, dev):
                        "streams": W.P, "rows": W.R,
                        "l2": "per-layer document KV and question rows exceed L2"},
             "doc_tflops": tfs, "doc_frac_of_sustained_bf16": tfs / world / peaks["bf16_sustained"],
-            "per_layer_us": {"doc_pass": durs["doc"] * 1e3, "suffix_merge": durs["suffix"] * 1e3,
+            "per_layer_us": {"doc_pass": durs["doc"] * 1e3, "question_part": durs["suffix"] * 1e3,
                              "doc_pass_tflops": doc_tfs,
                              "doc_pass_frac_burst_bf16": doc_tfs / peaks["bf16"],
                              "doc_pass_frac_sustained_bf16": doc_tfs / peaks["bf16_sustained"],
@@ -789,8 +789,9 @@ def load_peaks():
 
 
 def measure_doc_pass(step: DecodeStep, reps: int):
-    """Average device duration of the document-pass kernel and of the suffix
-    kernel, from CUDA events the library records around them on the
+    """Average device duration of the document-pass kernel and of what follows
+    it (the suffix kernel of a decode step; the run finding and question
+    kernel of a prefill), from CUDA events the library records around them on the
     launching stream.  The step with the events is captured as its own CUDA
     graph (event-record nodes), so host launch overhead cannot leak into the
     intervals; each replay re-records all 3 events of every layer."""
