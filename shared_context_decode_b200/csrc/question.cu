@@ -159,19 +159,32 @@ __global__ void __launch_bounds__(QCfg<D>::WARPS * 32, 1) question_attn(const QP
 
   const int n_runs = *p.n_runs;
   const int groups = (p.rows + kGroupRows - 1) / kGroupRows;
-  const int64_t tasks = (int64_t)n_runs * p.H;
-  const int64_t GW = (int64_t)gridDim.x * C::WARPS;
+  const int tasks = n_runs * p.H;
+  const int GW = gridDim.x * C::WARPS;
   const size_t seg_elems = (size_t)p.S_cap * D;
 
+  // The slots holding a row's document partials, c0 .. c1, depend only on
+  // the row's unit (head, row group): kept for the last unit seen, they are
+  // computed about once a task instead of twice a tile (two 64-bit
+  // divisions each).
+  int cu = -1, cc0 = 0, cc1 = -1;
+  const int64_t head_tiles = plan_head_tiles(p.plan);
+
   // task = head * n_runs + run: neighbouring warps share a head.  The next
-  // task's run record is loaded while this one runs.
-  int64_t task = (int64_t)blockIdx.x * C::WARPS + warp;
+  // task's run record is loaded while this one runs.  (The launch checks
+  // that rows * H fits in 32 bits.)
+  int task = blockIdx.x * C::WARPS + warp;
+  int run_n = task % max(n_runs, 1);
   int4 rec_n = make_int4(0, 0, 0, 0);
-  if (task < tasks) rec_n = p.runs[task % n_runs];
+  if (task < tasks) rec_n = p.runs[run_n];
   for (; task < tasks; task += GW) {
-    const int h = (int)(task / n_runs);
+    const int h = task / n_runs, run = task - h * n_runs;
     const int4 rec = rec_n;
-    if (task + GW < tasks) rec_n = p.runs[(task + GW) % n_runs];
+    if (task + GW < tasks) {
+      run_n = run + GW;  // (task + GW) mod n_runs without a division when GW < n_runs
+      if (run_n >= n_runs) run_n = (task + GW) % n_runs;
+      rec_n = p.runs[run_n];
+    }
     const int r_begin = rec.x, r_end = rec.y, s = rec.z, n = rec.w;
     const bool served = stream_query(s, p.P_max);
     if (h == 0 && lane == 0 && (s == 0 || s > p.P_max)) set_status(p.status, PP_DEV_BAD_STREAM);
@@ -251,9 +264,14 @@ __global__ void __launch_bounds__(QCfg<D>::WARPS * 32, 1) question_attn(const QP
         auto first = [&](int row, int& c0, int& c1, int64_t& sl0) {
           const int g = row / kGroupRows;
           const int u = h * groups + g;
-          const int64_t ub = plan_unit_begin(p.plan, u);
-          c0 = plan_cta_of(p.plan, ub);
-          c1 = plan_cta_of(p.plan, ub + plan_unit_tiles(p.plan, g) - 1);
+          if (u != cu) {  // first tile of unit u: h * (tiles of a head) + its groups' tiles
+            const int64_t ub = h * head_tiles + (p.plan.causal ? (int64_t)g * (g + 1) : (int64_t)g * p.plan.T);
+            cc0 = plan_cta_of(p.plan, ub);
+            cc1 = plan_cta_of(p.plan, ub + plan_unit_tiles(p.plan, g) - 1);
+            cu = u;
+          }
+          c0 = cc0;
+          c1 = cc1;
           sl0 = (int64_t)u * p.plan.max_chunks * kGroupRows + row % kGroupRows;
         };
         if (va) {
@@ -454,6 +472,7 @@ cudaError_t launch_question_attn(const pp_kv_layer& L, const uint16_t* q, const 
     }
     // at most rows runs: the grid covers rows * H tasks, persistent past it
     const int64_t tasks = (int64_t)rows * L.H;
+    if (tasks > 0x7fffffff - 2048LL * warps) return cudaErrorInvalidValue;  // task indexes are 32-bit
     int64_t ctas = (tasks + warps - 1) / warps;
     if (ctas > num_sms) ctas = num_sms;
     kernel<<<(int)ctas, warps * 32, smem, st>>>(prm);
