@@ -347,13 +347,15 @@ __global__ void __launch_bounds__(QCfg<D>::WARPS * 32, 1) question_attn(const QP
         cmb = fmaxf(cmb, __shfl_xor_sync(0xffffffffu, cmb, 2));
         const float nma = fmaxf(m_a, cma), nmb = fmaxf(m_b, cmb);
         const float ba = nma == -INFINITY ? 0.f : nma, bb = nmb == -INFINITY ? 0.f : nmb;
-        const float corr_a = exp2f(m_a - ba), corr_b = exp2f(m_b - bb);  // m = -inf gives 0
+        // MUFU exponentials, flush-to-zero: every argument is <= 0, so a result
+        // below 2^-126 only drops a probability far under the bf16 step
+        const float corr_a = ex2_mufu(m_a - ba), corr_b = ex2_mufu(m_b - bb);  // m = -inf gives 0
         float sa = 0.f, sb = 0.f;
         uint32_t pk[C::ST][2];  // probabilities as bf16 pairs: [nt][row a, row b]
 #pragma unroll
         for (int nt = 0; nt < C::ST; ++nt) {
-          const float p0 = exp2f(sc[nt][0] - ba), p1 = exp2f(sc[nt][1] - ba);
-          const float p2 = exp2f(sc[nt][2] - bb), p3 = exp2f(sc[nt][3] - bb);
+          const float p0 = ex2_mufu(sc[nt][0] - ba), p1 = ex2_mufu(sc[nt][1] - ba);
+          const float p2 = ex2_mufu(sc[nt][2] - bb), p3 = ex2_mufu(sc[nt][3] - bb);
           sa += p0 + p1;
           sb += p2 + p3;
           pk[nt][0] = f2_to_bf2(p0, p1);

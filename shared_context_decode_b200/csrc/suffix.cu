@@ -297,6 +297,11 @@ __global__ void __launch_bounds__(SufCfg<D, BAL>::WARPS * 32) suffix_merge(const
   // each segment is read once, so its lines go first and the document
   // partials the merge reads stay in L2
   const uint64_t pol = l2_policy_evict_first();
+  // The slots c0 .. c1 holding an item's document partials depend only on
+  // its unit (head, row group), which neighbouring items share: kept for the
+  // last unit seen (two 64-bit divisions saved per item).
+  int cu = -1, cc0 = 0, cc1 = -1;
+  const int64_t head_tiles = plan_head_tiles(p.plan);
   uint32_t issued = 0, consumed = 0;
   bool ok = true;
   for (int64_t k0 = 0; ok && k0 < n_w; k0 += C::TBL) {
@@ -403,10 +408,15 @@ __global__ void __launch_bounds__(SufCfg<D, BAL>::WARPS * 32) suffix_merge(const
       int64_t slot0 = 0;
       const int rr = r % kGroupRows;
       if (valid && p.has_doc) {
-        const int u = h * groups + r / kGroupRows;
-        const int64_t ub = plan_unit_begin(p.plan, u);
-        c0 = plan_cta_of(p.plan, ub);
-        c1 = plan_cta_of(p.plan, ub + plan_unit_tiles(p.plan, r / kGroupRows) - 1);
+        const int grp = r / kGroupRows, u = h * groups + grp;
+        if (u != cu) {  // a new unit (head, row group): its slots, once per unit, not per item
+          const int64_t ub = h * head_tiles + (p.plan.causal ? (int64_t)grp * (grp + 1) : (int64_t)grp * p.plan.T);
+          cc0 = plan_cta_of(p.plan, ub);
+          cc1 = plan_cta_of(p.plan, ub + plan_unit_tiles(p.plan, grp) - 1);
+          cu = u;
+        }
+        c0 = cc0;
+        c1 = cc1;
         slot0 = (int64_t)u * p.plan.max_chunks;
       }
       float2 pre_ml[C::PRE];
