@@ -270,8 +270,8 @@ pp_status pp_decode_attn_noalloc(const pp_kv_layer *layer, int32_t doc_len, cons
 /*
  * Workspace bytes pp_prefill_attn needs for R question rows: the document
  * pass's fp32 partial results (as for decode) and the question runs -- 16
- * bytes a row (whole groups of 256 rows) and their count -- which are
- * needed with or without a document.
+ * bytes a row (whole groups of 256 rows), their count and a task counter
+ * (one 256-byte block) -- which are needed with or without a document.
  */
 size_t pp_prefill_workspace_bytes(int32_t R, int32_t H, int32_t d, int32_t doc_len,
                                   const pp_options *opt);

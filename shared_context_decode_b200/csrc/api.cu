@@ -124,7 +124,7 @@ struct WsLayout {
 // row's stream length when the pass carries a decode step's append, and the
 // decode suffix pass's counters and partials for items cut between warps;
 // question prefill (questions = true): the question runs (at most one per
-// row) and their count.
+// row), their count and the question kernel's task counter.
 WsLayout ws_layout(const SplitPlan& p, int d, bool questions) {
   WsLayout w;
   const size_t slots = (size_t)p.units * p.max_chunks * pp::kGroupRows;
@@ -138,7 +138,7 @@ WsLayout ws_layout(const SplitPlan& p, int d, bool questions) {
   w.split_ml = w.split_o + up(2 * warps * d * sizeof(float));
   w.runs = w.split_ml + up(2 * warps * 2 * sizeof(float));
   w.n_runs = w.runs + (questions ? up((size_t)p.G * pp::kGroupRows * sizeof(int4)) : 0);
-  w.total = w.n_runs + (questions ? up(sizeof(int32_t)) : 0);
+  w.total = w.n_runs + (questions ? up(2 * sizeof(int32_t)) : 0);
   return w;
 }
 

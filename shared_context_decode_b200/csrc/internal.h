@@ -67,13 +67,14 @@ cudaError_t launch_doc_merge(int rows, int H, int d, const SplitPlan& plan, cons
                              uint16_t* o, float* lse, cudaStream_t st);
 // Question part of a prefill call: the runs of consecutive rows with one
 // stream id (one block; runs[k] = first row, end row, stream id, visible
-// segment keys), then one warp per (run, head) with the merge first.
+// segment keys; n_runs[0] = their count, n_runs[1] = 0 for the task
+// counter), then one warp per (run, head) with the merge first.
 cudaError_t launch_question_runs(const pp_kv_layer& L, const int16_t* q_sid, int rows, int4* runs,
                                  int32_t* n_runs, cudaStream_t st);
 cudaError_t launch_question_attn(const pp_kv_layer& L, const uint16_t* q, const int16_t* q_sid,
                                  const int32_t* q_pos, int rows, float scale, const SplitPlan& plan,
                                  bool has_doc, const Partials& part, uint16_t* o, float* lse,
-                                 const int4* runs, const int32_t* n_runs, int num_sms,
+                                 const int4* runs, int32_t* n_runs, int num_sms,
                                  cudaStream_t st);
 cudaError_t launch_visibility(const pp_kv_layer& L, int doc_len, const int16_t* q_sid,
                               const int32_t* q_pos, int nq, int32_t* count_out, uint8_t* mask_out,

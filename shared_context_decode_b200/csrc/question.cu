@@ -70,6 +70,7 @@ struct QParams {
   float* lse;
   const int4* runs;     // [n_runs] (first row, end row, stream id as given, visible segment keys)
   const int32_t* n_runs;
+  int32_t* next_task;   // tasks drawn past the first GW (zeroed by question_runs)
 };
 
 // Runs of consecutive rows with the same stream id, in row order.  One block;
@@ -126,7 +127,10 @@ __global__ void __launch_bounds__(1024) question_runs(const int16_t* __restrict_
   __syncthreads();
   for (int k = threadIdx.x; k < total; k += blockDim.x)
     runs[k].y = k + 1 < total ? runs[k + 1].x : rows;
-  if (threadIdx.x == 0) *n_runs = total;
+  if (threadIdx.x == 0) {
+    n_runs[0] = total;
+    n_runs[1] = 0;  // the question kernel's task counter
+  }
 }
 
 // Folds the partial (m2, l2, o2) of one row into (m, l, acc); o2 gives the
@@ -170,20 +174,31 @@ __global__ void __launch_bounds__(QCfg<D>::WARPS * 32, 1) question_attn(const QP
   int cu = -1, cc0 = 0, cc1 = -1;
   const int64_t head_tiles = plan_head_tiles(p.plan);
 
-  // task = head * n_runs + run: neighbouring warps share a head.  The next
-  // task's run record is loaded while this one runs.  (The launch checks
-  // that rows * H fits in 32 bits.)
+  // task = head * n_runs + run, so tasks taken in order share a head.  A
+  // warp's first task is its index; later ones come from a counter (zeroed
+  // by question_runs), each drawn a task ahead and its run record loaded
+  // while the task before it runs: a warp that drew short runs takes more of
+  // them, where fixed shares left the unluckiest warp half again the mean
+  // number of tiles.  (The launch checks that rows * H fits in 32 bits.)
+  auto draw = [&]() -> int {
+    int t = 0;
+    if (lane == 0) t = GW + atomicAdd(p.next_task, 1);
+    return __shfl_sync(0xffffffffu, t, 0);
+  };
   int task = blockIdx.x * C::WARPS + warp;
-  int run_n = task % max(n_runs, 1);
+  int task_n = tasks;
   int4 rec_n = make_int4(0, 0, 0, 0);
-  if (task < tasks) rec_n = p.runs[run_n];
-  for (; task < tasks; task += GW) {
-    const int h = task / n_runs, run = task - h * n_runs;
+  if (task < tasks) {
+    rec_n = p.runs[task % n_runs];
+    task_n = draw();
+  }
+  while (task < tasks) {
+    const int h = task / n_runs;
     const int4 rec = rec_n;
-    if (task + GW < tasks) {
-      run_n = run + GW;  // (task + GW) mod n_runs without a division when GW < n_runs
-      if (run_n >= n_runs) run_n = (task + GW) % n_runs;
-      rec_n = p.runs[run_n];
+    const int next = task_n;
+    if (next < tasks) {
+      rec_n = p.runs[next % n_runs];
+      task_n = draw();
     }
     const int r_begin = rec.x, r_end = rec.y, s = rec.z, n = rec.w;
     const bool served = stream_query(s, p.P_max);
@@ -423,6 +438,7 @@ __global__ void __launch_bounds__(QCfg<D>::WARPS * 32, 1) question_attn(const QP
     }
     if (nchunks > 0 && loaded >= 0) cp_async_wait_all();  // nothing in flight past the task
     __syncwarp();
+    task = next;
   }
 }
 
@@ -437,7 +453,7 @@ cudaError_t launch_question_runs(const pp_kv_layer& L, const int16_t* q_sid, int
 cudaError_t launch_question_attn(const pp_kv_layer& L, const uint16_t* q, const int16_t* q_sid,
                                  const int32_t* q_pos, int rows, float scale, const SplitPlan& plan,
                                  bool has_doc, const Partials& part, uint16_t* o, float* lse,
-                                 const int4* runs, const int32_t* n_runs, int num_sms,
+                                 const int4* runs, int32_t* n_runs, int num_sms,
                                  cudaStream_t st) {
   QParams prm;
   prm.q = q;
@@ -462,6 +478,7 @@ cudaError_t launch_question_attn(const pp_kv_layer& L, const uint16_t* q, const 
   prm.lse = lse;
   prm.runs = runs;
   prm.n_runs = n_runs;
+  prm.next_task = n_runs + 1;
   auto go = [&](auto kernel, int warps, int smem, std::atomic<uint64_t>& ready) -> cudaError_t {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
