@@ -178,8 +178,8 @@ __global__ void __launch_bounds__(QCfg<D>::WARPS * 32, 1) question_attn(const QP
   // warp's first task is its index; later ones come from a counter (zeroed
   // by question_runs), each drawn a task ahead and its run record loaded
   // while the task before it runs: a warp that drew short runs takes more of
-  // them, where fixed shares left the unluckiest warp half again the mean
-  // number of tiles.  (The launch checks that rows * H fits in 32 bits.)
+  // them instead of a fixed share of about seven tasks of 1-3 tiles.  (The
+  // launch checks that rows * H fits in 32 bits.)
   auto draw = [&]() -> int {
     int t = 0;
     if (lane == 0) t = GW + atomicAdd(p.next_task, 1);
