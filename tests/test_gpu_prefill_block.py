@@ -4,7 +4,8 @@ split into several runs), runs of many 16-row tiles over segments longer
 than one 48-key chunk, follow-up questions behind cached answers (rows whose
 segment holds earlier tokens), inactive and out-of-range rows inside runs,
 d = 64, no document, runs that cross a 256-row group of document partials,
-row counts that leave a ragged last tile.
+row counts that leave a ragged last tile, more (run, head) tasks than the
+kernel has warps with one workspace reused across calls.
 
 Visibility rule: project page "Read Once, Answer Many", section "How it
 works", item 1 -- a row sees the document and the tokens of its own stream
@@ -144,3 +145,35 @@ def test_rows_spanning_two_row_groups():
     layer, keys = build(H, d, N, seg, 32, seed=9)
     sid, pos = question_rows(seg, N)
     run(layer, keys, N, H, d, sid, pos, seed=9)
+
+
+def test_many_tasks_and_a_reused_workspace():
+    # 48 questions x 32 heads = 1536 (run, head) tasks, more than the
+    # question kernel's warps (8 per SM), so most warps draw further tasks
+    # from the counter in the workspace.  One workspace, filled with 0xff
+    # bytes first, serves two calls: each call starts its counter from zero,
+    # so both give the same bits, and they match the oracle.
+    m = gu.pp()
+    H, d, N = 32, 64, 200
+    seg = [int(x) for x in np.random.default_rng(11).integers(1, 40, size=48)]
+    layer, keys = build(H, d, N, seg, 40, seed=11)
+    sid, pos = question_rows(seg, N)
+    R = len(sid)
+    ws = m.workspace(m.prefill_workspace_bytes(R, H, d, N), DEV)
+    ws.fill_(255)
+    q = wl.randn_bf16((R, H, d), wl.seed_of("pfblock", "q", 11), DEV)
+    sid_t = torch.from_numpy(np.asarray(sid, np.int16)).to(DEV)
+    pos_t = torch.from_numpy(np.asarray(pos, np.int32)).to(DEV)
+    outs = []
+    for _ in range(2):
+        lse = torch.empty((R, H), dtype=torch.float32, device=DEV)
+        o = m.prefill_attn(layer, N, q, sid_t, pos_t, 0.11, lse=lse, ws=ws)
+        torch.cuda.synchronize()
+        assert m.device_status(layer) == 0
+        outs.append((o, lse))
+    assert torch.equal(outs[0][0], outs[1][0])
+    assert torch.equal(outs[0][1], outs[1][1])
+    k, v, kks, kkp = keys
+    ref_o, ref_lse, _ = oracle.masked_attention(bf16_bits(q), np.asarray(sid), np.asarray(pos),
+                                                k, v, kks, kkp, 0.11)
+    gu.compare(outs[1][0], outs[1][1], ref_o, ref_lse, "prefill, reused workspace")
