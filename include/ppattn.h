@@ -30,6 +30,10 @@
  *     default stream), perform no host synchronisation and no allocation,
  *     and may be captured into a CUDA graph -- except pp_get_device_status,
  *     which synchronises.
+ *   - A workspace holds one call's intermediate results (document partials,
+ *     counters); calls that may run at the same time (on different streams)
+ *     need separate workspaces.  Calls ordered on one stream may share one:
+ *     each call initialises what it reads.
  *   - Host-side argument checks return an error before anything is
  *     launched.  Errors found on the device set bits of the layer's device
  *     status word (PP_DEV_*), read with pp_get_device_status.
